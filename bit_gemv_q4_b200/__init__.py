@@ -1,0 +1,185 @@
+"""Python binding of libgq (include/gq.h): argument marshalling only.
+
+Every function below passes device pointers, sizes and the current CUDA stream
+to the C entry point of the same name and raises ``GQError`` on a non-OK
+status.  All arithmetic happens in the CUDA kernels of libgq.so; there is no
+Python or CPU fallback, and importing this package fails if the library has
+not been built (``python -m bit_gemv_q4_b200.build``).
+
+PyTorch is used only to allocate device memory and to name the stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgq.so")
+
+GQ_OK = 0
+GQ_F32, GQ_F16, GQ_BF16 = 0, 1, 2
+GQ_FMT_Q4_0, GQ_FMT_KSB = 0, 1
+GQ_DEV_NONFINITE, GQ_DEV_RANGE, GQ_DEV_TIMEOUT = 1, 2, 4
+GQ_GEMV_PDL = 1
+
+# every symbol include/gq.h declares
+EXPORTS = (
+    "gq_abi_version", "gq_status_string", "gq_status_from_dev",
+    "gq_q4_0_bytes", "gq_ksb_bytes",
+    "gq_quantize_q4_0", "gq_quantize_ksb",
+    "gq_dequantize_q4_0", "gq_dequantize_ksb",
+    "gq_gemv_q4_0", "gq_gemv_ksb",
+)
+
+_DTYPE_CODE = {torch.float32: GQ_F32, torch.float16: GQ_F16, torch.bfloat16: GQ_BF16}
+
+
+class GQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {gq_status_string(status)} (status {status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libgq.so not found at {LIB_PATH}; build it with `python -m bit_gemv_q4_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    i64, vp, c_int, c_uint = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_uint
+    L.gq_abi_version.restype = c_int
+    L.gq_status_string.argtypes = [c_int]
+    L.gq_status_string.restype = ctypes.c_char_p
+    L.gq_status_from_dev.argtypes = [c_int]
+    L.gq_status_from_dev.restype = c_int
+    L.gq_q4_0_bytes.argtypes = [i64]
+    L.gq_q4_0_bytes.restype = ctypes.c_size_t
+    L.gq_ksb_bytes.argtypes = [i64]
+    L.gq_ksb_bytes.restype = ctypes.c_size_t
+    for name in ("gq_quantize_q4_0", "gq_quantize_ksb"):
+        f = getattr(L, name)
+        f.argtypes = [vp, i64, vp, vp, vp]
+        f.restype = c_int
+    for name in ("gq_dequantize_q4_0", "gq_dequantize_ksb"):
+        f = getattr(L, name)
+        f.argtypes = [vp, i64, vp, vp]
+        f.restype = c_int
+    for name in ("gq_gemv_q4_0", "gq_gemv_ksb"):
+        f = getattr(L, name)
+        f.argtypes = [vp, i64, i64, vp, c_int, i64, vp, c_int, c_uint, vp, vp]
+        f.restype = c_int
+    return L
+
+
+lib = _load()
+
+
+def gq_abi_version() -> int:
+    return int(lib.gq_abi_version())
+
+
+def gq_status_string(status: int) -> str:
+    return lib.gq_status_string(int(status)).decode()
+
+
+def gq_status_from_dev(flags: int) -> int:
+    return int(lib.gq_status_from_dev(int(flags)))
+
+
+def gq_q4_0_bytes(n: int) -> int:
+    return int(lib.gq_q4_0_bytes(int(n)))
+
+
+def gq_ksb_bytes(n: int) -> int:
+    return int(lib.gq_ksb_bytes(int(n)))
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors passed to libgq must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libgq must be contiguous")
+    return t.data_ptr() or None
+
+
+def _check(status: int, where: str) -> None:
+    if status != GQ_OK:
+        raise GQError(status, where)
+
+
+def _quantize(name: str, nbytes, x: torch.Tensor, out, dev_status, stream):
+    if x.dtype != torch.float32:
+        raise TypeError("quantizer input must be float32")
+    n = x.numel()
+    if out is None:
+        out = torch.empty(max(nbytes(n), 0), dtype=torch.uint8, device=x.device)
+    _check(getattr(lib, name)(_ptr(x), n, _ptr(out), _ptr(dev_status), _stream(stream)), name)
+    return out
+
+
+def gq_quantize_q4_0(x: torch.Tensor, out: torch.Tensor | None = None,
+                     dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """fp32 values (numel % 32 == 0) -> uint8 Q4_0 blocks (18 bytes per 32)."""
+    return _quantize("gq_quantize_q4_0", gq_q4_0_bytes, x, out, dev_status, stream)
+
+
+def gq_quantize_ksb(x: torch.Tensor, out: torch.Tensor | None = None,
+                    dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """fp32 values (numel % 256 == 0) -> uint8 super-blocks (138 bytes per 256)."""
+    return _quantize("gq_quantize_ksb", gq_ksb_bytes, x, out, dev_status, stream)
+
+
+def _dequantize(name: str, q: torch.Tensor, n: int, out, stream):
+    if out is None:
+        out = torch.empty(n, dtype=torch.float32, device=q.device)
+    _check(getattr(lib, name)(_ptr(q), int(n), _ptr(out), _stream(stream)), name)
+    return out
+
+
+def gq_dequantize_q4_0(q: torch.Tensor, n: int, out: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    return _dequantize("gq_dequantize_q4_0", q, n, out, stream)
+
+
+def gq_dequantize_ksb(q: torch.Tensor, n: int, out: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    return _dequantize("gq_dequantize_ksb", q, n, out, stream)
+
+
+def _gemv(name: str, W: torch.Tensor, M: int, K: int, x: torch.Tensor, y_dtype, out,
+          flags: int, dev_status, stream):
+    x2 = x if x.dim() == 2 else x.reshape(1, -1)
+    B = x2.shape[0]
+    if x2.shape[1] != K:
+        raise ValueError(f"x has {x2.shape[1]} columns, expected K={K}")
+    if x2.dtype not in _DTYPE_CODE or y_dtype not in _DTYPE_CODE:
+        raise TypeError("activations and outputs must be float32, float16 or bfloat16")
+    if out is None:
+        out = torch.empty((B, M), dtype=y_dtype, device=x2.device)
+    _check(getattr(lib, name)(_ptr(W), int(M), int(K), _ptr(x2), _DTYPE_CODE[x2.dtype], B,
+                              _ptr(out), _DTYPE_CODE[out.dtype], int(flags), _ptr(dev_status),
+                              _stream(stream)), name)
+    return out
+
+
+def gq_gemv_q4_0(W: torch.Tensor, M: int, K: int, x: torch.Tensor, y_dtype=torch.float16,
+                 out: torch.Tensor | None = None, flags: int = 0,
+                 dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y[B, M] = W_hat[M, K] @ x[B, K]^T for Q4_0 weights; B in 1..8."""
+    return _gemv("gq_gemv_q4_0", W, M, K, x, y_dtype, out, flags, dev_status, stream)
+
+
+def gq_gemv_ksb(W: torch.Tensor, M: int, K: int, x: torch.Tensor, y_dtype=torch.float16,
+                out: torch.Tensor | None = None, flags: int = 0,
+                dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y[B, M] = W_hat[M, K] @ x[B, K]^T for super-block weights; B in 1..8."""
+    return _gemv("gq_gemv_ksb", W, M, K, x, y_dtype, out, flags, dev_status, stream)

@@ -1,0 +1,159 @@
+/*
+ * gq.h -- C ABI of libgq: GGUF-style 4-bit block weight quantization and the
+ * dequantize-fused matrix-vector / small-batch matrix products that stream
+ * those weights, as hand-written CUDA for sm_100a (NVIDIA B200).
+ *
+ * Formats (byte layouts are normative):
+ *
+ *   Q4_0 -- "GGUF 量化内幕 第4章：Q4_0 块量化格式解析", sections 4.1.2 and 4.2.1.
+ *     32 weights in 18 bytes: bytes 0-1 the FP16 scale d (little-endian bit
+ *     pattern), bytes 2-17 qs[0..15]; qs[j] holds the 4-bit code of weight j
+ *     in its low nibble and of weight j+16 in its high nibble.  4.5 bits per
+ *     weight.  Decoding (section 4.2.2 / 4.3): w = d * (code - 8).
+ *
+ *   KSB (super-block K-quant) -- "GGUF K-quants" (hugo-blog), section "套娃"
+ *     and its bits table.  256 weights in 138 bytes: bytes 0-1 the FP16
+ *     super-scale S, bytes 2-9 the INT8 sub-scales q_0..q_7, then 8 x 16 bytes
+ *     of codes; sub-block j (weights 32j..32j+31) has its 16 code bytes at
+ *     offset 10+16j with the Q4_0 low/high nibble split.  4.3125 bits per
+ *     weight.  Decoding: w = (S * q_j) * (code - 8); both products are exact
+ *     in fp32, so decoded values are bit-exact whatever the evaluation order.
+ *
+ *   Matrices: W has M rows of K weights; each row is quantized along K and its
+ *   blocks are stored contiguously, rows one after another (row m starts at
+ *   byte m * gq_q4_0_bytes(K) or m * gq_ksb_bytes(K)).
+ *
+ * Quantization rule (the pages leave the rounding open; this library fixes
+ * it): d = FP16(absmax / 7) with an IEEE fp32 quotient rounded to nearest even
+ * in FP16; code = clamp(rint(x / d) + 8, 0, 15) with an IEEE fp32 quotient and
+ * rint rounding half to even; d == 0 gives code 8.  For KSB each sub-block's
+ * d_j is formed this way, then S = FP16(max_j d_j / 127) (the post's
+ * (max - (-max)) / (127 - (-127))), q_j = clamp(rint(d_j / S), 0, 127)
+ * (0 when S == 0), and the codes are taken against the rebuilt scale S * q_j.
+ *
+ * Conventions shared by every entry point:
+ *   - All data pointers are device (or managed) memory owned by the caller;
+ *     the library allocates nothing and keeps no pointer after returning.
+ *   - `stream` is a cudaStream_t passed as void* (NULL: the legacy default
+ *     stream).  Every call is asynchronous on that stream; a returned GQ_OK
+ *     means the arguments were valid and the launch was accepted.
+ *   - Argument checks are synchronous and happen before any launch: on any
+ *     error nothing is launched and nothing is written.
+ *   - Data-dependent problems are reported through the optional device word
+ *     `dev_status` (int*, may be NULL): the kernels atomically OR GQ_DEV_*
+ *     bits into it; the caller zeroes it beforehand and reads it after the
+ *     stream is synchronized (gq_status_from_dev() maps it to a gq_status).
+ *     No kernel traps or asserts.
+ *   - Base pointers must be 16-byte aligned (GQ_ERR_ALIGNMENT otherwise).
+ *     Packed weights are read in whole 16-byte granules: bytes after the end
+ *     of a packed buffer, up to the next 16-byte boundary, may be read and are
+ *     ignored (such a granule never crosses a page, so this cannot fault).
+ *   - Sizes of 0 are valid and launch nothing (a K of 0 writes y = 0).
+ */
+#ifndef GQ_H
+#define GQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GQ_API __attribute__((visibility("default")))
+#else
+#define GQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GQ_ABI_VERSION 1
+
+typedef enum gq_status {
+    GQ_OK = 0,
+    GQ_ERR_INVALID_ARG = 1,  /* NULL pointer, negative size, bad enum      */
+    GQ_ERR_SHAPE = 2,        /* size not a whole number of blocks, B range  */
+    GQ_ERR_ALIGNMENT = 3,    /* pointer not 16-byte aligned                 */
+    GQ_ERR_DTYPE = 4,        /* unsupported element type                    */
+    GQ_ERR_NONFINITE = 5,    /* (device) NaN or infinity in quantizer input */
+    GQ_ERR_RANGE = 6,        /* (device) a scale overflowed FP16            */
+    GQ_ERR_TIMEOUT = 7,      /* (device) a bounded wait in a kernel gave up */
+    GQ_ERR_CUDA = 8,         /* a CUDA launch or runtime call failed        */
+    GQ_ERR_WORKSPACE = 9     /* workspace missing or too small              */
+} gq_status;
+
+typedef enum gq_dtype { GQ_F32 = 0, GQ_F16 = 1, GQ_BF16 = 2 } gq_dtype;
+typedef enum gq_format { GQ_FMT_Q4_0 = 0, GQ_FMT_KSB = 1 } gq_format;
+
+/* Bits ORed into *dev_status by the kernels. */
+#define GQ_DEV_NONFINITE 1
+#define GQ_DEV_RANGE     2
+#define GQ_DEV_TIMEOUT   4
+
+/* gq_gemv_* flags.
+ * GQ_GEMV_PDL: launch with programmatic dependent launch.  The kernel may be
+ *   scheduled while the previous kernel on the stream is still running; it
+ *   streams W at once and waits for that kernel to finish before it reads x
+ *   or writes y.  Use it only when W is not written by work still in flight
+ *   on the stream (the usual case in decode, where weights are static). */
+#define GQ_GEMV_PDL 1u
+
+GQ_API int gq_abi_version(void);
+GQ_API const char* gq_status_string(int status);
+/* First error among the GQ_DEV_* bits of a device status word (GQ_OK if 0). */
+GQ_API gq_status gq_status_from_dev(int dev_flags);
+
+/* Packed bytes of n weights; 0 when n < 0 or n is not a whole number of
+ * blocks (32 for Q4_0, 256 for KSB).  Q4_0 chapter 4.1.2: 18 bytes / 32;
+ * K-quants bits table: 138 bytes / 256. */
+GQ_API size_t gq_q4_0_bytes(int64_t n);
+GQ_API size_t gq_ksb_bytes(int64_t n);
+
+/* Quantize n fp32 values into Q4_0 blocks (Q4_0 chapter 4.4 for the shape of
+ * the step, with this library's rounding rule above).
+ *   x:   n floats, 16-byte aligned.  n % 32 == 0 (GQ_ERR_SHAPE otherwise).
+ *   out: gq_q4_0_bytes(n) bytes, 16-byte aligned.
+ *   dev_status: optional; GQ_DEV_NONFINITE if any input is NaN/inf (that
+ *     block's bytes are then unspecified), GQ_DEV_RANGE if absmax/7 rounds to
+ *     an FP16 infinity (the block then stores d = inf and codes 8). */
+GQ_API gq_status gq_quantize_q4_0(const float* x, int64_t n, void* out,
+                                  int* dev_status, void* stream);
+
+/* Quantize n fp32 values into KSB super-blocks (K-quants post, "套娃": the
+ * eight sub-block scales are quantized to INT8 against an FP16 super-scale).
+ *   n % 256 == 0; out holds gq_ksb_bytes(n) bytes.  dev_status as above. */
+GQ_API gq_status gq_quantize_ksb(const float* x, int64_t n, void* out,
+                                 int* dev_status, void* stream);
+
+/* Decode n weights to fp32 (Q4_0 chapter 4.3: y = d * (code - 8); K-quants
+ * post step 5: the INT8 sub-scale times S rebuilds the scale).  Output values
+ * are exact, hence identical on every implementation.
+ *   q: packed bytes (16-byte aligned); out: n floats (16-byte aligned). */
+GQ_API gq_status gq_dequantize_q4_0(const void* q, int64_t n, float* out, void* stream);
+GQ_API gq_status gq_dequantize_ksb(const void* q, int64_t n, float* out, void* stream);
+
+/* Dequantize-fused matrix-vector product for decode, y = W_hat * x, for a
+ * batch of 1..8 activation vectors (the matrix multiply that consumes the
+ * decoded weights: Q4_0 chapter 4.3; the memory-bound decode step: the
+ * TurboQuant W4A8 post, section 2.3).
+ *   W: M x K packed (row layout above), 16-byte aligned.  K % 32 == 0 (Q4_0)
+ *      or K % 256 == 0 (KSB).  M <= 2^31 - 1, K <= 2^24.
+ *   x: [B][K] of x_dtype (GQ_F16, GQ_BF16 or GQ_F32), row-major.
+ *   y: [B][M] of y_dtype (GQ_F16, GQ_BF16 or GQ_F32), row-major.
+ *   B: 1..8 (0 launches nothing).
+ * Arithmetic: products of the exact decoded weights with the exact inputs
+ * (fp32 x is split exactly into three bfloat16 terms), accumulated in fp32,
+ * rounded once to y_dtype.  flags: 0 or GQ_GEMV_PDL.  dev_status: optional,
+ * receives GQ_DEV_TIMEOUT if a pipeline wait ever gives up. */
+GQ_API gq_status gq_gemv_q4_0(const void* W, int64_t M, int64_t K,
+                              const void* x, int x_dtype, int64_t B,
+                              void* y, int y_dtype, unsigned flags,
+                              int* dev_status, void* stream);
+GQ_API gq_status gq_gemv_ksb(const void* W, int64_t M, int64_t K,
+                             const void* x, int x_dtype, int64_t B,
+                             void* y, int y_dtype, unsigned flags,
+                             int* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GQ_H */

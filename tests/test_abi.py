@@ -1,0 +1,114 @@
+"""The C-ABI library on the CPU: it loads, exports every entry point that
+include/gq.h declares, and rejects bad arguments synchronously with the
+documented status before touching the GPU.  Nothing here launches a kernel:
+every call below fails validation (fake device addresses are never touched).
+"""
+import os
+import re
+import subprocess
+
+import pytest
+
+import bit_gemv_q4_b200 as gq
+from conftest import ROOT
+
+GQ_OK, INVALID, SHAPE, ALIGN, DTYPE = 0, 1, 2, 3, 4
+A = 0x10000000  # 16-byte-aligned fake device address (never dereferenced)
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "gq.h")).read()
+    return sorted(set(re.findall(r"GQ_API\s+[\w\s\*]+?\b(gq_\w+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    decl = declared_symbols()
+    assert len(decl) >= 11
+    assert set(decl) == set(gq.EXPORTS)
+    out = subprocess.run(["nm", "-D", "--defined-only", gq.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (gq_\w+)", out))
+    assert set(decl) <= exported
+    # nothing but the declared entry points leaks out of the library
+    assert exported == set(decl)
+
+
+def test_version_and_status_strings():
+    assert gq.gq_abi_version() == 1
+    for s in range(10):
+        assert gq.gq_status_string(s)
+    assert gq.gq_status_from_dev(0) == GQ_OK
+    assert gq.gq_status_from_dev(gq.GQ_DEV_RANGE) == 6
+    assert gq.gq_status_from_dev(gq.GQ_DEV_NONFINITE | gq.GQ_DEV_RANGE) == 5
+    assert gq.gq_status_from_dev(gq.GQ_DEV_TIMEOUT | gq.GQ_DEV_RANGE) == 7
+
+
+def test_sizes():
+    assert gq.gq_q4_0_bytes(32) == 18 and gq.gq_q4_0_bytes(4096 * 11008) == 4096 * 344 * 18
+    assert gq.gq_ksb_bytes(256) == 138 and gq.gq_ksb_bytes(11008 * 4096) == 11008 * 16 * 138
+    for bad in (-32, 31, 48):
+        assert gq.gq_q4_0_bytes(bad) == 0
+    for bad in (-256, 32, 288):
+        assert gq.gq_ksb_bytes(bad) == 0
+    assert gq.gq_q4_0_bytes(0) == 0 and gq.gq_ksb_bytes(0) == 0
+
+
+@pytest.mark.parametrize("name,block", [("gq_quantize_q4_0", 32), ("gq_quantize_ksb", 256)])
+def test_quantize_validation(name, block):
+    f = getattr(gq.lib, name)
+    assert f(A, -block, A, None, None) == INVALID
+    assert f(A, block + 1, A, None, None) == SHAPE
+    assert f(A, block // 2, A, None, None) == SHAPE
+    assert f(None, 0, None, None, None) == GQ_OK          # empty: no launch
+    assert f(None, block, A, None, None) == INVALID
+    assert f(A, block, None, None, None) == INVALID
+    assert f(A + 4, block, A, None, None) == ALIGN
+    assert f(A, block, A + 2, None, None) == ALIGN
+    assert f(A, block, A, A + 1, None) == ALIGN          # dev_status must be int-aligned
+
+
+@pytest.mark.parametrize("name,block", [("gq_dequantize_q4_0", 32), ("gq_dequantize_ksb", 256)])
+def test_dequantize_validation(name, block):
+    f = getattr(gq.lib, name)
+    assert f(A, -1, A, None) == INVALID
+    assert f(A, block + 32 if block == 256 else 33, A, None) == SHAPE
+    assert f(None, 0, None, None) == GQ_OK
+    assert f(None, block, A, None) == INVALID
+    assert f(A + 8, block, A, None) == ALIGN
+    assert f(A, block, A + 12, None) == ALIGN
+
+
+@pytest.mark.parametrize("name,block", [("gq_gemv_q4_0", 32), ("gq_gemv_ksb", 256)])
+def test_gemv_validation(name, block):
+    f = getattr(gq.lib, name)
+    K = 4 * block
+    ok = dict(W=A, M=64, K=K, x=A, xt=1, B=1, y=A, yt=1, flags=0, st=None, s=None)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["W"], a["M"], a["K"], a["x"], a["xt"], a["B"], a["y"], a["yt"], a["flags"],
+                 a["st"], a["s"])
+
+    assert call(M=-1) == INVALID
+    assert call(K=-block) == INVALID
+    assert call(B=-1) == INVALID
+    assert call(xt=7) == DTYPE
+    assert call(yt=-1) == DTYPE
+    assert call(flags=2) == INVALID
+    assert call(K=K + 16) == SHAPE
+    assert call(B=9) == SHAPE
+    assert call(K=1 << 25) == SHAPE
+    assert call(M=0) == GQ_OK and call(B=0) == GQ_OK     # empty: no launch
+    assert call(y=None) == INVALID
+    assert call(W=None) == INVALID
+    assert call(x=None) == INVALID
+    assert call(W=A + 2) == ALIGN
+    assert call(x=A + 8) == ALIGN
+    assert call(y=A + 4) == ALIGN
+    assert call(st=A + 2) == ALIGN
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        gq.gq_quantize_q4_0(torch.zeros(64))

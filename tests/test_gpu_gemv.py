@@ -1,0 +1,125 @@
+"""GPU dequantize-fused GEMV against the oracle's fp64 product.
+
+Tolerance, per output: |y - y_ref| <= 1e-4 * sum_k |w_hat||x| plus one unit in
+the last place of the output type (the fp32 result is rounded once to fp16 /
+bf16).  Weights are quantized by the oracle, so every input byte of the GPU
+product comes from the oracle side."""
+import numpy as np
+import pytest
+import torch
+
+import bit_gemv_q4_b200 as gq
+import oracle
+import synth
+from gpu_helpers import KSB, Q40, assert_product_close, x_for_oracle
+
+pytestmark = pytest.mark.gpu
+
+_cache = {}
+
+
+def packed(fmt, M, K, gen="gauss", seed=None):
+    key = (fmt, M, K, gen, seed)
+    if key not in _cache:
+        s = (M * 7 + K) if seed is None else seed
+        w = (synth.gaussian_weights if gen == "gauss" else synth.logstd_weights)(M, K, seed=s)
+        q, _ = oracle.quantize(fmt, w.numpy().ravel())
+        _cache[key] = q
+    return _cache[key]
+
+
+def run_gemv(fmt, q, M, K, x, ydt, flags=0):
+    f = gq.gq_gemv_q4_0 if fmt == Q40 else gq.gq_gemv_ksb
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = f(torch.from_numpy(q).cuda(), M, K, x.cuda(), y_dtype=ydt, flags=flags, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    return y
+
+
+def check(fmt, M, K, B, xdt, ydt, gen="gauss", flags=0, seed=None):
+    q = packed(fmt, M, K, gen, seed)
+    x = synth.activations(B, K, seed=B + K, dtype=xdt)
+    y = run_gemv(fmt, q, M, K, x, ydt, flags)
+    xo, xt = x_for_oracle(x)
+    Y, bound = oracle.gemm(fmt, q, M, K, xo, xt)
+    return assert_product_close(y, Y, bound)
+
+
+# the five workloads' product shapes
+def test_tiny_fp32_in_fp32_out():
+    # W 256x1024 (seed 0) N(0, 0.02^2) with 0.1 % x10 outliers; x fp32; y fp32
+    check(Q40, 256, 1024, 1, torch.float32, torch.float32, seed=0)
+
+
+def test_decode_4096x4096_fp16():
+    check(Q40, 4096, 4096, 1, torch.float16, torch.float16)
+
+
+@pytest.mark.parametrize("B", [1, 8])
+def test_ksb_mlp_11008x4096(B):
+    check(KSB, 11008, 4096, B, torch.float16, torch.float16, gen="logstd")
+
+
+@pytest.mark.parametrize("fmt", [Q40, KSB])
+@pytest.mark.parametrize("M,K", [(4096, 11008), (11008, 4096)])
+def test_metric_shapes(fmt, M, K):
+    # both orientations of the 4096x11008 headline shape, with and without PDL
+    check(fmt, M, K, 1, torch.float16, torch.float16)
+    check(fmt, M, K, 1, torch.float16, torch.float16, flags=gq.GQ_GEMV_PDL)
+
+
+# edge shapes: ragged row tiles, single blocks, K chunks with ragged tails
+@pytest.mark.parametrize("fmt,M,K", [
+    (Q40, 1, 32), (Q40, 7, 64), (Q40, 17, 288), (Q40, 33, 1056), (Q40, 4097, 2080),
+    (Q40, 5, 3072 + 32), (KSB, 1, 256), (KSB, 15, 512), (KSB, 17, 1280), (KSB, 129, 2304),
+])
+def test_edge_shapes(fmt, M, K):
+    check(fmt, M, K, 1, torch.float16, torch.float16)
+
+
+@pytest.mark.parametrize("B", [1, 2, 3, 5, 7, 8])
+@pytest.mark.parametrize("xdt", [torch.float16, torch.bfloat16, torch.float32])
+def test_batches_and_dtypes(B, xdt):
+    ydt = {torch.float16: torch.float32, torch.bfloat16: torch.bfloat16,
+           torch.float32: torch.float16}[xdt]
+    check(Q40, 100, 2048, B, xdt, ydt)
+    check(KSB, 100, 2048, B, xdt, ydt, gen="logstd")
+
+
+def test_wide_batch_window():
+    # B=8 with K=11008: the activations do not fit shared memory at once and
+    # are streamed in windows
+    check(Q40, 64, 11008, 8, torch.float32, torch.float32)
+    check(KSB, 48, 11008, 8, torch.float16, torch.float32)
+
+
+def test_k_zero_writes_zeros():
+    y = torch.full((2, 5), 7.0, device="cuda")
+    W = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    x = torch.zeros((2, 0), dtype=torch.float16, device="cuda")
+    gq.gq_gemv_q4_0(W, 5, 0, x, y_dtype=torch.float32, out=y)
+    torch.cuda.synchronize()
+    assert torch.all(y == 0)
+
+
+def test_constant_codes_closed_form():
+    # every block d = 0.5, every code 11 -> y = 1.5 * sum(x)
+    M, K = 40, 4096
+    blk = np.array([0x00, 0x38] + [0xBB] * 16, np.uint8)
+    q = np.tile(blk, M * K // 32)
+    x = synth.activations(3, K, seed=3, dtype=torch.float16)
+    y = run_gemv(Q40, q, M, K, x, torch.float32)
+    want = 1.5 * x.double().sum(dim=1)
+    assert torch.allclose(y.double().cpu(), want[:, None].expand(3, M), rtol=1e-5, atol=1e-4)
+
+
+def test_misaligned_rows_large_k():
+    # K = 11008 super-blocks give 5934-byte rows, so most rows start off a
+    # 16-byte boundary; an offset view of W shifts them all
+    M, K = 40, 11008
+    q = packed(KSB, M, K)
+    x = synth.activations(1, K, seed=1, dtype=torch.float16)
+    y = run_gemv(KSB, q, M, K, x, torch.float32)
+    Y, bound = oracle.gemm(KSB, q, M, K, *x_for_oracle(x))
+    assert_product_close(y, Y, bound)

@@ -1,0 +1,149 @@
+"""GPU quantize / dequantize against the oracle, byte for byte and bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import bit_gemv_q4_b200 as gq
+import oracle
+import synth
+from gpu_helpers import KSB, Q40
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_quantize(fmt, w: torch.Tensor):
+    x = w.reshape(-1).float().contiguous().cuda()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    f = gq.gq_quantize_q4_0 if fmt == Q40 else gq.gq_quantize_ksb
+    q = f(x, dev_status=st)
+    torch.cuda.synchronize()
+    return q.cpu().numpy(), int(st.item())
+
+
+def gpu_dequantize(fmt, q: np.ndarray, n: int):
+    f = gq.gq_dequantize_q4_0 if fmt == Q40 else gq.gq_dequantize_ksb
+    out = f(torch.from_numpy(q).cuda(), n)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def assert_bytes_equal(got, want, blk):
+    if not np.array_equal(got, want):
+        diff = np.nonzero(got != want)[0]
+        b = diff[0] // blk
+        raise AssertionError(f"{diff.size} bytes differ; first in block {b}: gpu "
+                             f"{got[b * blk:(b + 1) * blk].tolist()} oracle "
+                             f"{want[b * blk:(b + 1) * blk].tolist()}")
+
+
+CASES = [
+    # (format, rows, cols, generator) -- the five workloads' shapes plus ragged tails
+    (Q40, 256, 1024, "gauss"),     # tiny workload (seed 0)
+    (Q40, 1, 32, "gauss"),         # one block
+    (Q40, 67, 32, "gauss"),        # 67 blocks: ragged CTA tile
+    (Q40, 4096, 4096, "gauss"),    # decode shape
+    (Q40, 11008, 4096, "logstd"),
+    (KSB, 256, 1024, "gauss"),
+    (KSB, 1, 256, "gauss"),
+    (KSB, 9, 256, "logstd"),       # ragged CTA tile
+    (KSB, 11008, 4096, "logstd"),  # MLP shape
+    (KSB, 4096, 11008, "gauss"),
+]
+
+
+@pytest.mark.parametrize("fmt,M,K,gen", CASES)
+def test_quantize_bit_exact(fmt, M, K, gen):
+    seed = 0 if (M, K) == (256, 1024) else M + K
+    w = (synth.gaussian_weights if gen == "gauss" else synth.logstd_weights)(M, K, seed=seed)
+    got, st = gpu_quantize(fmt, w)
+    want, flags = oracle.quantize(fmt, w.numpy().ravel())
+    assert st == 0 and flags == 0
+    assert_bytes_equal(got, want, 18 if fmt == Q40 else 138)
+
+
+@pytest.mark.parametrize("fmt", [Q40, KSB])
+def test_dequantize_bit_exact(fmt):
+    # oracle-made blocks, plus arbitrary byte patterns with finite scales
+    w = synth.logstd_weights(333, 512, seed=5)
+    q, _ = oracle.quantize(fmt, w.numpy().ravel())
+    n = w.numel()
+    assert np.array_equal(gpu_dequantize(fmt, q, n).view(np.uint32),
+                          oracle.dequantize(fmt, q, n).view(np.uint32))
+    rng = np.random.default_rng(1)
+    blk = 18 if fmt == Q40 else 138
+    nb = 4099 if fmt == Q40 else 515
+    r = rng.integers(0, 256, size=nb * blk, dtype=np.uint8).reshape(nb, blk)
+    r[:, 1] &= 0x7B  # keep the FP16 scale finite
+    q = r.ravel().copy()
+    n = nb * (32 if fmt == Q40 else 256)
+    assert np.array_equal(gpu_dequantize(fmt, q, n).view(np.uint32),
+                          oracle.dequantize(fmt, q, n).view(np.uint32))
+
+
+def _edge_blocks():
+    rows = []
+    rows.append(np.zeros(32))                                   # all zero
+    x = np.zeros(32); x[3] = 7 * 2.0 ** -20; x[20] = -3 * 2.0 ** -20
+    rows.append(x)                                              # subnormal FP16 scale
+    x = np.zeros(32); x[:14] = (np.arange(-7, 7) + 0.5) * 0.25; x[14] = 1.75
+    rows.append(x)                                              # exact ties
+    rows.append(np.array([0.01 * (i - 15) / 15 for i in range(31)] + [10.0]))  # outlier demo
+    x = np.zeros(32); x[5] = -1e-30
+    rows.append(x)                                              # scale underflows to 0
+    x = np.linspace(-3e4, 3e4, 32)
+    rows.append(x)                                              # large but in range
+    x = np.full(32, -0.0)
+    rows.append(x)
+    return np.concatenate(rows).astype(np.float32)
+
+
+@pytest.mark.parametrize("fmt", [Q40, KSB])
+def test_quantize_edge_blocks(fmt):
+    x = _edge_blocks()
+    if fmt == KSB:
+        x = np.concatenate([x, np.zeros(256 - x.size % 256, np.float32)])
+    got, st = gpu_quantize(fmt, torch.from_numpy(x))
+    want, flags = oracle.quantize(fmt, x)
+    assert st == flags == 0
+    assert_bytes_equal(got, want, 18 if fmt == Q40 else 138)
+
+
+@pytest.mark.parametrize("fmt", [Q40, KSB])
+def test_quantize_status_flags(fmt):
+    n = 32 * 64 if fmt == Q40 else 256 * 8
+    x = np.zeros(n, np.float32)
+    x[40] = 7 * 70000.0      # absmax/7 overflows FP16 -> range
+    _, st = gpu_quantize(fmt, torch.from_numpy(x))
+    _, flags = oracle.quantize(fmt, x)
+    assert st == flags == gq.GQ_DEV_RANGE
+    x[40] = 1.0
+    x[300] = np.nan
+    _, st = gpu_quantize(fmt, torch.from_numpy(x))
+    assert st & gq.GQ_DEV_NONFINITE
+    assert gq.gq_status_from_dev(st) == 5
+
+
+@pytest.mark.parametrize("fmt", [Q40, KSB])
+def test_quantize_1e9_sampled(fmt):
+    """Quantize of 1e9 fp32 weights N(0, 0.02^2) generated on the device (the
+    throughput workload); a random sample of blocks is checked byte for byte
+    against the oracle on the same input values."""
+    n = 1_000_000_000
+    rows = n // 8000
+    w = synth.gaussian_weights(rows, 8000, seed=4, frac=0.0, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    f = gq.gq_quantize_q4_0 if fmt == Q40 else gq.gq_quantize_ksb
+    q = f(w.view(-1), dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    blk_w, blk_b = (32, 18) if fmt == Q40 else (256, 138)
+    nblk = n // blk_w
+    rng = np.random.default_rng(9)
+    pick = np.unique(np.concatenate([rng.integers(0, nblk, 3000), [0, nblk - 1]]))
+    idx = torch.from_numpy(pick).cuda()
+    xin = w.view(-1, blk_w)[idx].cpu().numpy()
+    got = q.view(-1, blk_b)[idx].cpu().numpy()
+    want, _ = oracle.quantize(fmt, xin.ravel())
+    assert_bytes_equal(got.ravel(), want, blk_b)
+    del w, q
+    torch.cuda.empty_cache()
