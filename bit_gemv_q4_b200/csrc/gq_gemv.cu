@@ -6,30 +6,34 @@
 // memory-bound decode setting (TurboQuant W4A8 post, section 2.3).
 //
 // Design (sm_100a):
-//  * One CTA owns 16 consecutive rows (one m16 MMA tile) over all of K.  Its
-//    rows are contiguous in HBM, so the CTA reads one contiguous byte range.
-//  * Warp 0 is the producer: for each K chunk of 1024 weights it issues one
-//    1-D bulk async copy (cp.async.bulk, no multicast) per row into a 4-stage
-//    shared-memory ring, completion tracked by mbarrier transaction counts.
-//    Row pieces need not be 16-byte aligned (18-byte / 138-byte blocks): the
-//    copy covers the enclosing 16-byte granules and consumers index from the
-//    piece's offset inside its first granule.
-//  * Warps 1..4 consume: each takes a quarter of the chunk, decodes 4-bit
-//    codes straight into MMA A fragments (code - 8 exactly, by exponent-bias
-//    tricks on packed halves), and runs warp MMA m16n8k16 with fp32
-//    accumulation.  The batch columns are the MMA's N dimension (N = 8 covers
-//    B <= 8; B = 1 replicates one column).  Because every block has its own
-//    scale, the two MMAs of a 32-weight block accumulate into a fresh
-//    fragment that is then scaled and added in fp32 -- products are exact
-//    (4-bit integer x fp16/bf16), so no weight is ever rounded.
-//  * fp32 activations are split exactly into three bfloat16 terms (three
-//    MMAs per k-step); fp16 and bf16 activations use one.
-//  * The activations live in shared memory in the fragment order of the MMA
-//    B operand; a warp reads its B fragments with one 16-byte load per block.
-//  * Programmatic dependent launch: the producer streams W immediately;
-//    consumers wait for the preceding grid before reading x or writing y.
-//  * Every mbarrier wait is bounded; on expiry the kernel sets
-//    GQ_DEV_TIMEOUT, drains its own in-flight copies (bounded) and exits.
+//  * Work unit: a group of 16 consecutive rows (one m16 MMA tile) over all of
+//    K.  The rows of a group are contiguous in HBM.  CTAs are persistent and
+//    take groups g = blockIdx.x, blockIdx.x + gridDim.x, ...
+//  * Warp 0 produces: for each K chunk of 1024 weights of a group it issues
+//    one 1-D bulk async copy (cp.async.bulk, no multicast) per row into a
+//    6-stage shared-memory ring, completion tracked by mbarrier transaction
+//    counts, running ahead across group boundaries.  Row pieces need not be
+//    16-byte aligned (18-byte / 138-byte blocks): a copy covers the enclosing
+//    16-byte granules and consumers index from the piece's offset.
+//  * Warps 1..8 consume: each takes an eighth of every chunk, decodes the
+//    4-bit codes straight into MMA A fragments (code - 8, exactly, by
+//    exponent-bias tricks on packed halves) and runs warp MMA m16n8k16 with
+//    fp32 accumulation.  Batch columns are the MMA's N dimension (N = 8
+//    covers B <= 8; with B = 1 every column holds the same vector).  Each
+//    block has its own scale, so the two MMAs of a 32-weight block write a
+//    fresh fragment that is scaled and added in fp32: all products are exact
+//    (4-bit integer x fp16/bf16), no weight is ever rounded.
+//  * When every row starts on a 16-byte boundary (Q4_0 with K % 256 == 0,
+//    ksb with K % 2048 == 0) all byte offsets inside a stage are known at
+//    compile time; otherwise they are taken per row at run time.
+//  * fp32 activations are split exactly into three bfloat16 terms (three MMAs
+//    per k-step); fp16 and bf16 activations use one.  Activations sit in
+//    shared memory in B-fragment order (one 16-byte load per lane per block)
+//    and are loaded once per CTA when they fit, else per window.
+//  * Programmatic dependent launch: the producer streams W at once; consumers
+//    wait for the preceding grid before reading x or writing y.
+//  * Every wait is bounded; on expiry the kernel sets GQ_DEV_TIMEOUT, drains
+//    its own in-flight copies (bounded) and exits.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -42,16 +46,35 @@
 namespace gq {
 namespace {
 
-constexpr int kRows = 16;                           // rows per CTA
-constexpr int kConsumers = 4;                       // consumer warps
+#ifndef GQ_GEMV_CHUNK
+#define GQ_GEMV_CHUNK 2048
+#endif
+#ifndef GQ_GEMV_STAGES
+#define GQ_GEMV_STAGES 4
+#endif
+
+#ifndef GQ_GEMV_CONSUMERS
+#define GQ_GEMV_CONSUMERS 8
+#endif
+#ifndef GQ_GEMV_MINB
+#define GQ_GEMV_MINB 2
+#endif
+
+constexpr int kRows = 16;                           // rows per group (MMA M)
+constexpr int kConsumers = GQ_GEMV_CONSUMERS;       // consumer warps
 constexpr int kThreads = 32 * (1 + kConsumers);
-constexpr int kChunkW = 1024;                       // weights per row per stage
-constexpr int kPitch = 592;                         // bytes per row slot (>= 590)
+constexpr int kChunkW = GQ_GEMV_CHUNK;              // weights per row per stage
+constexpr int kSubPerWarp = kChunkW / 32 / kConsumers;  // 32-weight blocks per warp
+// bytes per row slot: the row piece plus up to 14 bytes of leading offset,
+// rounded to 16, and chosen so that rows r = 0..7 fall on distinct banks
+constexpr int kPitch = (kChunkW == 1024) ? 592 : 1168;
 constexpr int kStageBytes = kRows * kPitch + 16;    // +16: window-read slack
-constexpr int kStages = 4;
+constexpr int kStages = GQ_GEMV_STAGES;
 constexpr int kXBlk = 64;                           // B-fragment bytes per 32 weights
 constexpr int kXStride = (kChunkW / 32) * kXBlk + 64;  // per (chunk, batch row), padded
-constexpr int kXSmemMax = 96 * 1024;                // activation window budget
+constexpr int kXSmemMax = 72 * 1024;                // activation window budget
+static_assert(kChunkW == 1024 || kChunkW == 2048, "supported chunk sizes");
+static_assert(kSubPerWarp % 2 == 0, "blocks per warp come in pairs");
 
 enum { XT_F16 = 0, XT_BF16 = 1, XT_F32 = 2 };
 
@@ -73,7 +96,7 @@ struct GemvArgs {
   void* y;
   int* dev_status;
   long long budget;
-  int B, ytype, nchunks, win;  // win: chunks per activation window
+  int B, ytype, nchunks, win, ngroups;  // win: chunks per activation window
 };
 
 // ---- decode 8 codes (one 32-bit word = qs[4t..4t+3]) into four A registers
@@ -82,19 +105,18 @@ struct GemvArgs {
 //   r2 = (w[4t+1],  w[4t+3])     r3 = (w[4t+17], w[4t+19])
 // fp16: 0x6400 | n is 1024 + n; 0x6400 | (n << 4) is 1024 + 16n.
 __device__ __forceinline__ void decode_f16(uint32_t q, uint32_t r[4]) {
-  const uint32_t q8 = q >> 8;
-  __half2 h0, h1, h2, h3;
+  const uint32_t q8 = __umulhi(q, 0x01000000u);  // q >> 8, on the FMA pipe
   uint32_t t0 = lop3_and_or(q, 0x000F000Fu, 0x64006400u);
   uint32_t t1 = lop3_and_or(q, 0x00F000F0u, 0x64006400u);
   uint32_t t2 = lop3_and_or(q8, 0x000F000Fu, 0x64006400u);
   uint32_t t3 = lop3_and_or(q8, 0x00F000F0u, 0x64006400u);
-  const __half2 k1032 = __float2half2_rn(1032.0f);
-  const __half2 k16th = __float2half2_rn(0.0625f);
-  const __half2 km72 = __float2half2_rn(-72.0f);
-  h0 = __hsub2(*reinterpret_cast<__half2*>(&t0), k1032);
-  h1 = __hfma2(*reinterpret_cast<__half2*>(&t1), k16th, km72);
-  h2 = __hsub2(*reinterpret_cast<__half2*>(&t2), k1032);
-  h3 = __hfma2(*reinterpret_cast<__half2*>(&t3), k16th, km72);
+  const __half2 k1032 = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
+  const __half2 k16th = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
+  const __half2 km72 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));
+  __half2 h0 = __hsub2(*reinterpret_cast<__half2*>(&t0), k1032);
+  __half2 h1 = __hfma2(*reinterpret_cast<__half2*>(&t1), k16th, km72);
+  __half2 h2 = __hsub2(*reinterpret_cast<__half2*>(&t2), k1032);
+  __half2 h3 = __hfma2(*reinterpret_cast<__half2*>(&t3), k16th, km72);
   r[0] = *reinterpret_cast<uint32_t*>(&h0);
   r[1] = *reinterpret_cast<uint32_t*>(&h1);
   r[2] = *reinterpret_cast<uint32_t*>(&h2);
@@ -103,7 +125,8 @@ __device__ __forceinline__ void decode_f16(uint32_t q, uint32_t r[4]) {
 
 // bf16: 0x4300 | n is 128 + n (7 mantissa bits, so nibbles are shifted down).
 __device__ __forceinline__ void decode_bf16(uint32_t q, uint32_t r[4]) {
-  const __nv_bfloat162 k136 = __float2bfloat162_rn(136.0f);
+  const __nv_bfloat162 k136 =
+      __halves2bfloat162(__ushort_as_bfloat16(0x4308), __ushort_as_bfloat16(0x4308));
   uint32_t t[4];
   t[0] = lop3_and_or(q, 0x000F000Fu, 0x43004300u);
   t[1] = lop3_and_or(q >> 4, 0x000F000Fu, 0x43004300u);
@@ -116,113 +139,285 @@ __device__ __forceinline__ void decode_bf16(uint32_t q, uint32_t r[4]) {
   }
 }
 
-template <int XT>
-__device__ __forceinline__ void decode(uint32_t q, uint32_t r[4]) {
-  if constexpr (XT == XT_F16)
-    decode_f16(q, r);
-  else
-    decode_bf16(q, r);
+// The dynamic shared-memory array of every kernel in this file.  Loads below
+// index it by 32-bit byte offsets, so they are plain shared-memory loads with
+// immediate offsets, ordered after the stage's mbarrier wait.
+extern __shared__ __align__(128) uint8_t smem[];
+
+__device__ __forceinline__ uint32_t ld32(uint32_t off) {
+  return *reinterpret_cast<const uint32_t*>(smem + off);
+}
+__device__ __forceinline__ uint32_t ld16(uint32_t off) {
+  return *reinterpret_cast<const uint16_t*>(smem + off);
+}
+__device__ __forceinline__ uint4 ld128(uint32_t off) {
+  return *reinterpret_cast<const uint4*>(smem + off);
+}
+// four bytes at an offset that is 2 mod 4 (MIS == 2) or 0 mod 4 (MIS == 0)
+template <int MIS>
+__device__ __forceinline__ uint32_t ld32_at(uint32_t off) {
+  if constexpr (MIS == 0) {
+    return ld32(off);
+  } else {
+    return __byte_perm(ld32(off - 2), ld32(off + 2), 0x5432u);
+  }
+}
+// four bytes at an even offset whose alignment is known only at run time
+__device__ __forceinline__ uint32_t ld32_even(uint32_t off) {
+  const uint32_t b = off & ~3u;
+  return __byte_perm(ld32(b), ld32(b + 4), (off & 2u) ? 0x5432u : 0x3210u);
 }
 
+// One 32-weight block for rows r (codes qa) and r+8 (codes qb): both k16
+// MMAs over every activation term, into a fresh fragment c.
 template <int XT>
-__device__ __forceinline__ void mma(float c[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                    uint32_t a3, uint32_t b0, uint32_t b1) {
-  if constexpr (XT == XT_F16)
-    mma_f16(c, a0, a1, a2, a3, b0, b1);
-  else
-    mma_bf16(c, a0, a1, a2, a3, b0, b1);
-}
-
-// One 32-weight block for rows r (codes qa) and r+8 (codes qb): the two k16
-// MMAs of the block, over all activation terms, into c (zeroed by caller).
-template <int XT>
-__device__ __forceinline__ void block_mma(float c[4], uint32_t qa, uint32_t qb, uint32_t xaddr,
+__device__ __forceinline__ void block_mma(float c[4], uint32_t qa, uint32_t qb, uint32_t xp,
                                           uint32_t term_stride) {
   constexpr int kTerms = (XT == XT_F32) ? 3 : 1;
   uint32_t ra[4], rb[4];
-  decode<XT>(qa, ra);
-  decode<XT>(qb, rb);
+  if constexpr (XT == XT_F16) {
+    decode_f16(qa, ra);
+    decode_f16(qb, rb);
+    const uint4 xv = ld128(xp);
+    mma_f16_z(c, ra[0], rb[0], ra[2], rb[2], xv.x, xv.y);
+    mma_f16(c, ra[1], rb[1], ra[3], rb[3], xv.z, xv.w);
+  } else {
+    decode_bf16(qa, ra);
+    decode_bf16(qb, rb);
 #pragma unroll
-  for (int tm = 0; tm < kTerms; ++tm) {
-    const uint4 xv = lds128(xaddr + tm * term_stride);
-    // A regs: (row r, k lo) (row r+8, k lo) (row r, k hi) (row r+8, k hi)
-    mma<XT>(c, ra[0], rb[0], ra[2], rb[2], xv.x, xv.y);
-    mma<XT>(c, ra[1], rb[1], ra[3], rb[3], xv.z, xv.w);
+    for (int tm = 0; tm < kTerms; ++tm) {
+      const uint4 xv = ld128(xp + tm * term_stride);
+      if (tm == 0)
+        mma_bf16_z(c, ra[0], rb[0], ra[2], rb[2], xv.x, xv.y);
+      else
+        mma_bf16(c, ra[0], rb[0], ra[2], rb[2], xv.x, xv.y);
+      mma_bf16(c, ra[1], rb[1], ra[3], rb[3], xv.z, xv.w);
+    }
   }
 }
 
-// Load one window of activations into shared memory in B-fragment order.
-// For 32 weights of batch row b, lane-group t (0..3) reads 16 bytes:
-//   x[4t], x[4t+2], x[4t+1], x[4t+3], x[4t+16], x[4t+18], x[4t+17], x[4t+19]
-template <int XT>
-__device__ void load_x_window(uint8_t* xs, const void* x, int64_t K, int B, int c0, int nwin,
-                              uint32_t term_stride, int tid) {
-  const int64_t k_begin = static_cast<int64_t>(c0) * kChunkW;
-  const int64_t k_end = i64min(K, k_begin + static_cast<int64_t>(nwin) * kChunkW);
-  const int per_row = static_cast<int>((k_end - k_begin) / 8);
-  for (int idx = tid; idx < B * per_row; idx += 32 * kConsumers) {
-    const int b = idx / per_row;
-    const int k8 = (idx - b * per_row) * 8;  // relative to the window
-    const int64_t gk = k_begin + k8;
-    float v[8];
-    uint16_t bits[8];
-    if constexpr (XT == XT_F32) {
-      const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(x) + b * K + gk);
-      const float4 u0 = p[0], u1 = p[1];
-      v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
-      v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
-    } else {
-      const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + b * K + gk);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+// Scale a block's fragment and accumulate: acc[i] += d(row) * c[i].  With one
+// activation vector every column of c holds the same value; only columns 0
+// of rows r and r+8 are kept.
+template <bool NB1>
+__device__ __forceinline__ void scale_acc(float acc[4], const float c[4], float d0, float d1) {
+  acc[0] = fmaf(d0, c[0], acc[0]);
+  acc[2] = fmaf(d1, c[2], acc[2]);
+  if constexpr (!NB1) {
+    acc[1] = fmaf(d0, c[1], acc[1]);
+    acc[3] = fmaf(d1, c[3], acc[3]);
+  }
+}
+
+// ---------------------------------------------------------------- Q4_0 body
+// Block j of a stage: its two rows' code words and scales.
+template <bool ALIGNED, int J>
+__device__ __forceinline__ void q40_load(uint32_t row0, uint32_t row1, int t, int jb,
+                                         uint32_t& qa, uint32_t& qb, float& da, float& db) {
+  const uint32_t a = row0 + jb * 18;
+  const uint32_t b = row1 + jb * 18;
+  if constexpr (ALIGNED) {
+    // rows start on 16-byte boundaries and jb has the parity of J: the codes
+    // of an even block start 2 mod 4, of an odd block 0 mod 4
+    qa = ld32_at<(J & 1) ? 0 : 2>(a + 2 + 4 * t);
+    qb = ld32_at<(J & 1) ? 0 : 2>(b + 2 + 4 * t);
+  } else {
+    qa = ld32_even(a + 2 + 4 * t);
+    qb = ld32_even(b + 2 + 4 * t);
+  }
+  da = half_bits_to_float(ld16(a));
+  db = half_bits_to_float(ld16(b));
+}
+
+// A consumer warp's blocks w*kSubPerWarp .. +kSubPerWarp-1 of one stage.  A
+// full share is unrolled without branches -- every load is issued before the
+// first decode -- so the warp keeps many loads and MMAs in flight.
+template <int XT, bool NB1, bool ALIGNED>
+__device__ __forceinline__ void q40_chunk(float acc[4], uint32_t row0, uint32_t row1,
+                                          uint32_t xw, uint32_t term_stride, int w, int t,
+                                          int nvalid) {
+  const int jw = w * kSubPerWarp;  // even
+  if (nvalid >= kSubPerWarp) {
+    uint32_t qa[kSubPerWarp], qb[kSubPerWarp];
+    float da[kSubPerWarp], db[kSubPerWarp];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        bits[2 * i] = static_cast<uint16_t>(w[i] & 0xFFFFu);
-        bits[2 * i + 1] = static_cast<uint16_t>(w[i] >> 16);
-      }
+    for (int j = 0; j < kSubPerWarp; j += 2) {
+      q40_load<ALIGNED, 0>(row0, row1, t, jw + j, qa[j], qb[j], da[j], db[j]);
+      q40_load<ALIGNED, 1>(row0, row1, t, jw + j + 1, qa[j + 1], qb[j + 1], da[j + 1], db[j + 1]);
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int kk = k8 + i;
-      const int cw = kk / kChunkW, blk = (kk % kChunkW) / 32, p = kk % 32;
-      const int hi = p >> 4, pp = p & 15, t = pp >> 2, ii = pp & 3;
-      const int slot = hi * 4 + ((ii & 1) << 1) + (ii >> 1);
-      uint8_t* dst = xs + (cw * B + b) * kXStride + blk * kXBlk + t * 16 + slot * 2;
-      if constexpr (XT == XT_F32) {
+    for (int j = 0; j < kSubPerWarp; ++j) {
+      float c[4];
+      block_mma<XT>(c, qa[j], qb[j], xw + (jw + j) * kXBlk, term_stride);
+      scale_acc<NB1>(acc, c, da[j], db[j]);
+    }
+  } else {
+    // ragged last chunk of a row
+    for (int j = 0; j < nvalid; ++j) {
+      uint32_t qa, qb;
+      float da, db;
+      q40_load<false, 0>(row0, row1, t, jw + j, qa, qb, da, db);
+      float c[4];
+      block_mma<XT>(c, qa, qb, xw + (jw + j) * kXBlk, term_stride);
+      scale_acc<NB1>(acc, c, da, db);
+    }
+  }
+}
+
+// ----------------------------------------------------------------- ksb body
+// A consumer warp's kSubPerWarp sub-blocks of one super-block of the stage.
+// s~_j = S * q_j is applied as q_j per sub-block and S once at the end.  All
+// loads are issued before the first decode.
+template <int XT, bool NB1>
+__device__ __forceinline__ void ksb_chunk(float acc[4], uint32_t row0, uint32_t row1,
+                                          uint32_t xw, uint32_t term_stride, int w, int t) {
+  const int sb = (w * kSubPerWarp) >> 3, j0 = (w * kSubPerWarp) & 7;
+  const uint32_t a = row0 + sb * 138;
+  const uint32_t b = row1 + sb * 138;
+  const float Sa = half_bits_to_float(ld16(a));
+  const float Sb = half_bits_to_float(ld16(b));
+  uint32_t qja[2], qjb[2];
+  qja[0] = ld32_even(a + 2 + j0);
+  qjb[0] = ld32_even(b + 2 + j0);
+  if constexpr (kSubPerWarp > 4) {
+    qja[1] = ld32_even(a + 6 + j0);
+    qjb[1] = ld32_even(b + 6 + j0);
+  }
+  float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+  constexpr int kBatch = kSubPerWarp < 4 ? kSubPerWarp : 4;
+#pragma unroll
+  for (int h = 0; h < kSubPerWarp; h += kBatch) {  // batches of up to four sub-blocks
+    uint32_t na[kBatch], nb[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      na[j] = ld32_even(a + 10 + 16 * (j0 + h + j) + 4 * t);
+      nb[j] = ld32_even(b + 10 + 16 * (j0 + h + j) + 4 * t);
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      float c[4];
+      block_mma<XT>(c, na[j], nb[j], xw + (8 * sb + j0 + h + j) * kXBlk, term_stride);
+      const int q = h + j;  // sub-block index within this warp's share
+      const float fa = static_cast<float>(static_cast<int8_t>((qja[q >> 2] >> (8 * (q & 3))) & 0xFFu));
+      const float fb = static_cast<float>(static_cast<int8_t>((qjb[q >> 2] >> (8 * (q & 3))) & 0xFFu));
+      scale_acc<NB1>(sacc, c, fa, fb);
+    }
+  }
+  acc[0] = fmaf(Sa, sacc[0], acc[0]);
+  acc[2] = fmaf(Sb, sacc[2], acc[2]);
+  if constexpr (!NB1) {
+    acc[1] = fmaf(Sa, sacc[1], acc[1]);
+    acc[3] = fmaf(Sb, sacc[3], acc[3]);
+  }
+}
+
+// ---------------------------------------------------- activation windows
+// Load activations [k_begin, k_end) of all batch rows into shared memory in
+// B-fragment order: for each 32 weights and lane-group t (0..3), 16 bytes
+//   x[4t], x[4t+2], x[4t+1], x[4t+3], x[4t+16], x[4t+18], x[4t+17], x[4t+19]
+// Each thread moves 8 consecutive values as two 8-byte stores per term.
+template <int XT>
+__device__ __forceinline__ void store_x8(uint8_t* xs, const void* xsrc, int B, int b, int k8,
+                                         uint32_t term_stride, const uint4* raw) {
+  static_assert((kChunkW & (kChunkW - 1)) == 0, "chunk is a power of two");
+  const int cw = k8 / kChunkW, blk = (k8 & (kChunkW - 1)) >> 5, p = k8 & 31;
+  const int hi = p >> 4, t0 = (p & 15) >> 2;
+  // lane-group t0 gets (v0 v2 v1 v3) at slot 4*hi, lane-group t0+1 the next four
+  uint8_t* dst = xs + (cw * B + b) * kXStride + blk * kXBlk + t0 * 16 + hi * 8;
+  if constexpr (XT == XT_F32) {
+    const float v[8] = {__uint_as_float(raw[0].x), __uint_as_float(raw[0].y),
+                        __uint_as_float(raw[0].z), __uint_as_float(raw[0].w),
+                        __uint_as_float(raw[1].x), __uint_as_float(raw[1].y),
+                        __uint_as_float(raw[1].z), __uint_as_float(raw[1].w)};
+    uint32_t term[3][4];  // per term: bf16 pairs (v0,v1)(v2,v3)(v4,v5)(v6,v7)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t parts[3][2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
         // exact split v = b1 + b2 + b3 into bfloat16 terms
-        const __nv_bfloat16 b1 = __float2bfloat16_rn(v[i]);
-        const float r1 = __fsub_rn(v[i], __bfloat162float(b1));
+        const float vv = v[2 * i + h];
+        const __nv_bfloat16 b1 = __float2bfloat16_rn(vv);
+        const float r1 = __fsub_rn(vv, __bfloat162float(b1));
         const __nv_bfloat16 b2 = __float2bfloat16_rn(r1);
         const float r2 = __fsub_rn(r1, __bfloat162float(b2));
         const __nv_bfloat16 b3 = __float2bfloat16_rn(r2);
-        *reinterpret_cast<__nv_bfloat16*>(dst) = b1;
-        *reinterpret_cast<__nv_bfloat16*>(dst + term_stride) = b2;
-        *reinterpret_cast<__nv_bfloat16*>(dst + 2 * term_stride) = b3;
-      } else {
-        *reinterpret_cast<uint16_t*>(dst) = bits[i];
+        parts[0][h] = __bfloat16_as_ushort(b1);
+        parts[1][h] = __bfloat16_as_ushort(b2);
+        parts[2][h] = __bfloat16_as_ushort(b3);
+      }
+#pragma unroll
+      for (int tm = 0; tm < 3; ++tm) term[tm][i] = parts[tm][0] | (parts[tm][1] << 16);
+    }
+#pragma unroll
+    for (int tm = 0; tm < 3; ++tm) {
+      uint8_t* d = dst + tm * term_stride;
+      *reinterpret_cast<uint2*>(d) = make_uint2(__byte_perm(term[tm][0], term[tm][1], 0x5410),
+                                                __byte_perm(term[tm][0], term[tm][1], 0x7632));
+      *reinterpret_cast<uint2*>(d + 16) = make_uint2(__byte_perm(term[tm][2], term[tm][3], 0x5410),
+                                                     __byte_perm(term[tm][2], term[tm][3], 0x7632));
+    }
+  } else {
+    const uint4 u = raw[0];
+    *reinterpret_cast<uint2*>(dst) = make_uint2(__byte_perm(u.x, u.y, 0x5410), __byte_perm(u.x, u.y, 0x7632));
+    *reinterpret_cast<uint2*>(dst + 16) = make_uint2(__byte_perm(u.z, u.w, 0x5410), __byte_perm(u.z, u.w, 0x7632));
+  }
+}
+
+// Load activations [k_begin, k_end) of all batch rows into shared memory in
+// B-fragment order: for each 32 weights and lane-group t (0..3), 16 bytes
+//   x[4t], x[4t+2], x[4t+1], x[4t+3], x[4t+16], x[4t+18], x[4t+17], x[4t+19]
+// Each thread moves groups of 8 consecutive values; the global loads of four
+// groups are issued together before any of them is stored.
+template <int XT>
+__device__ void load_x_window(uint8_t* xs, const void* x, int64_t K, int B, int c0, int nwin,
+                              uint32_t term_stride, int tid) {
+  constexpr int kVec = (XT == XT_F32) ? 2 : 1;  // uint4 per 8 values
+  constexpr int kBatch = 4;
+  constexpr int kStride = 32 * kConsumers;
+  const int64_t k_begin = static_cast<int64_t>(c0) * kChunkW;
+  const int per_row = static_cast<int>((i64min(K, k_begin + static_cast<int64_t>(nwin) * kChunkW) - k_begin) / 8);
+  for (int b = 0; b < B; ++b) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(x) +
+                                                      (b * K + k_begin) * (XT == XT_F32 ? 4 : 2));
+    for (int base = tid; base < per_row; base += kBatch * kStride) {
+      uint4 raw[kBatch][kVec];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const int g8 = base + i * kStride;
+        if (g8 < per_row) {
+#pragma unroll
+          for (int v = 0; v < kVec; ++v) raw[i][v] = src[g8 * kVec + v];
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const int g8 = base + i * kStride;
+        if (g8 < per_row) store_x8<XT>(xs, x, B, b, g8 * 8, term_stride, raw[i]);
       }
     }
   }
 }
 
-template <int FMT, int XT>
-__global__ void __launch_bounds__(kThreads) gemv_kernel(const GemvArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
+template <int FMT, int XT, bool NB1, bool ALIGNED>
+__global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB) gemv_kernel(const GemvArgs a) {
   constexpr int kBlkW = Fmt<FMT>::kBlkW, kBlkB = Fmt<FMT>::kBlkB;
   constexpr int kTerms = (XT == XT_F32) ? 3 : 1;
+  constexpr int kBlkPerChunk = kChunkW / kBlkW;
+  constexpr int kChunkBytes = kBlkPerChunk * kBlkB;
 
   uint8_t* stages = smem;
   uint8_t* xs = smem + kStages * kStageBytes;
   const uint32_t term_stride = static_cast<uint32_t>(a.win * a.B * kXStride);
-  float* red = reinterpret_cast<float*>(xs + kTerms * term_stride);  // [kConsumers][32][4]
-  uint64_t* full = reinterpret_cast<uint64_t*>(red + kConsumers * 32 * 4);
+  float* red = reinterpret_cast<float*>(xs + kTerms * term_stride);  // [2][kConsumers][32][4]
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + 2 * kConsumers * 32 * 4);
   uint64_t* empty = full + kStages;
   uint64_t* cbar = empty + kStages;  // consumer-group barrier (bounded waits)
   int* abort_flag = reinterpret_cast<int*>(cbar + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kRows;
-  const int64_t nblk_row = a.K / kBlkW;
-  constexpr int kBlkPerChunk = kChunkW / kBlkW;
+  const int nblk_row = static_cast<int>(a.K / kBlkW);
+  const int nfull = nblk_row / kBlkPerChunk;  // chunks with every block present
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -239,51 +434,52 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(const GemvArgs a) {
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     const uint64_t pol = policy_evict_first();
-    int issued = 0;
+    int issued = 0;      // stage uses issued so far (all groups)
+    int s = 0;           // stage of the next use
+    uint32_t ph = 0;     // its phase parity
     bool ok = true;
-    for (int c = 0; c < a.nchunks && ok; ++c) {
-      const int s = c % kStages;
-      const uint32_t ph = static_cast<uint32_t>(c / kStages) & 1u;
-      if (!mbar_wait(&empty[s], ph ^ 1u, a.budget)) {
-        ok = false;
-        break;
-      }
-      if (*reinterpret_cast<volatile int*>(abort_flag)) {
-        ok = false;
-        break;
-      }
-      const int64_t b0 = static_cast<int64_t>(c) * kBlkPerChunk;
-      const int64_t nb = i64min(kBlkPerChunk, nblk_row - b0);
-      uint32_t len = 0;
-      const uint8_t* src_al = nullptr;
-      if (lane < kRows && m0 + lane < a.M) {
-        const uintptr_t src = reinterpret_cast<uintptr_t>(a.W) +
-                              static_cast<uintptr_t>((m0 + lane) * a.rowbytes + b0 * kBlkB);
-        const uintptr_t lo = src & ~static_cast<uintptr_t>(15);
-        const uintptr_t hi = (src + static_cast<uintptr_t>(nb * kBlkB) + 15) & ~static_cast<uintptr_t>(15);
-        src_al = reinterpret_cast<const uint8_t*>(lo);
-        len = static_cast<uint32_t>(hi - lo);
-      }
-      uint32_t total = len;
+    const uint32_t tail_bytes = static_cast<uint32_t>((nblk_row - nfull * kBlkPerChunk) * kBlkB);
+    for (int g = blockIdx.x; g < a.ngroups && ok; g += gridDim.x) {
+      const int64_t m0 = static_cast<int64_t>(g) * kRows;
+      const bool row_ok = lane < kRows && m0 + lane < a.M;
+      uintptr_t src = reinterpret_cast<uintptr_t>(a.W) +
+                      static_cast<uintptr_t>((m0 + (row_ok ? lane : 0)) * a.rowbytes);
+      for (int c = 0; c < a.nchunks; ++c, ++issued, src += kChunkBytes) {
+        if (!mbar_wait(&empty[s], ph ^ 1u, a.budget) ||
+            *reinterpret_cast<volatile int*>(abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint32_t nbytes = (c < nfull) ? static_cast<uint32_t>(kChunkBytes) : tail_bytes;
+        uint32_t len = 0;
+        uintptr_t lo = 0;
+        if (row_ok) {
+          lo = src & ~static_cast<uintptr_t>(15);
+          len = static_cast<uint32_t>(((src + nbytes + 15) & ~static_cast<uintptr_t>(15)) - lo);
+        }
+        uint32_t total = len;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xFFFFFFFFu, total, o);
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], total);
-      __syncwarp();
-      if (len) bulk_g2s(stages + s * kStageBytes + lane * kPitch, src_al, len, &full[s], pol);
-      issued = c + 1;
-    }
-    if (!ok) {
-      if (lane == 0) {
-        report(a.dev_status, GQ_DEV_TIMEOUT);
-        *reinterpret_cast<volatile int*>(abort_flag) = 1;
+        for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xFFFFFFFFu, total, o);
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], total);
+        __syncwarp();
+        if (len)
+          bulk_g2s(stages + s * kStageBytes + lane * kPitch, reinterpret_cast<const void*>(lo), len,
+                   &full[s], pol);
+        if (++s == kStages) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
+    }
+    if (!ok && lane == 0) {
+      report(a.dev_status, GQ_DEV_TIMEOUT);
+      *reinterpret_cast<volatile int*>(abort_flag) = 1;
     }
     // Drain: every issued copy must land before this CTA's shared memory is
     // released, whatever the consumers did.
     if (lane == 0) {
-      for (int c = max(0, issued - kStages); c < issued; ++c) {
-        const int s = c % kStages;
-        if (!mbar_wait(&full[s], static_cast<uint32_t>(c / kStages) & 1u, a.budget)) {
+      for (int u = max(0, issued - kStages); u < issued; ++u) {
+        if (!mbar_wait(&full[u % kStages], static_cast<uint32_t>(u / kStages) & 1u, a.budget)) {
           report(a.dev_status, GQ_DEV_TIMEOUT);
           break;
         }
@@ -293,13 +489,10 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(const GemvArgs a) {
   }
 
   // -------------------------------------------------------------- consumers
-  const int cw = warp - 1;                // consumer index 0..3
-  const int ctid = threadIdx.x - 32;      // 0..127
+  const int cw = warp - 1;                // consumer index 0..7
+  const int ctid = threadIdx.x - 32;      // 0..255
   const int r = lane >> 2, t = lane & 3;  // fragment row group / thread in group
   const int bsel = min(r, a.B - 1);       // batch column this lane's B fragment reads
-  const uint32_t stages_addr = smem_addr(stages);
-  const uint32_t xs_addr = smem_addr(xs);
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
   bool ok = true;
   uint32_t cphase = 0;
   // All consumer warps pass the same sequence of group barriers; a barrier is
@@ -312,153 +505,169 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(const GemvArgs a) {
     return done;
   };
 
+  // this warp's share of a ragged last chunk
+  int tail_valid;
+  if constexpr (FMT == GQ_FMT_Q4_0)
+    tail_valid = min(max(nblk_row - nfull * kBlkPerChunk - kSubPerWarp * cw, 0), kSubPerWarp);
+  else
+    tail_valid = ((cw * kSubPerWarp) >> 3) < nblk_row - nfull * kBlkPerChunk;
+
   pdl_wait();  // the preceding grid has finished: x is ready, y may be written
 
-  for (int c = 0; c < a.nchunks; ++c) {
-    if (c % a.win == 0) {
-      if (!group_sync()) {
+  const bool x_resident = (a.win >= a.nchunks);
+  if (x_resident) {
+    load_x_window<XT>(xs, a.x, a.K, a.B, 0, a.win, term_stride, ctid);
+    ok = group_sync();
+  }
+  const uint32_t x_chunk = static_cast<uint32_t>(a.B * kXStride);
+  const uint32_t x_lane = static_cast<uint32_t>(xs - smem) + bsel * kXStride + t * 16;
+
+  int s = 0;        // stage of the next use
+  uint32_t ph = 0;  // its phase parity
+  int gi = 0;       // groups done by this CTA
+  for (int g = blockIdx.x; g < a.ngroups && ok; g += gridDim.x, ++gi) {
+    const int64_t m0 = static_cast<int64_t>(g) * kRows;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    // offset of row r's (and r+8's) first byte inside its 16-byte granule
+    uint32_t off0 = static_cast<uint32_t>(
+        (reinterpret_cast<uintptr_t>(a.W) + static_cast<uintptr_t>((m0 + r) * a.rowbytes)) & 15u);
+    uint32_t off1 = static_cast<uint32_t>(
+        (reinterpret_cast<uintptr_t>(a.W) + static_cast<uintptr_t>((m0 + r + 8) * a.rowbytes)) & 15u);
+    uint32_t xw = x_lane;
+    int cw_in_win = 0;
+    for (int c = 0; c < a.nchunks; ++c) {
+      if (!x_resident && cw_in_win == 0) {
+        if (!group_sync()) { ok = false; break; }
+        load_x_window<XT>(xs, a.x, a.K, a.B, c, a.win, term_stride, ctid);
+        if (!group_sync()) { ok = false; break; }
+        xw = x_lane;
+      }
+      if (!mbar_wait(&full[s], ph, a.budget) || *reinterpret_cast<volatile int*>(abort_flag)) {
         ok = false;
         break;
       }
-      load_x_window<XT>(xs, a.x, a.K, a.B, c, a.win, term_stride, ctid);
-      if (!group_sync()) {
-        ok = false;
-        break;
+      const uint32_t stg = static_cast<uint32_t>(s * kStageBytes);  // stages start at offset 0
+      const bool whole = c < nfull;
+      if constexpr (FMT == GQ_FMT_Q4_0) {
+        const int nvalid = whole ? kSubPerWarp : tail_valid;
+        if constexpr (ALIGNED) {
+          q40_chunk<XT, NB1, true>(acc, stg + r * kPitch, stg + (r + 8) * kPitch, xw, term_stride,
+                                   cw, t, nvalid);
+        } else {
+          q40_chunk<XT, NB1, false>(acc, stg + r * kPitch + off0, stg + (r + 8) * kPitch + off1,
+                                    xw, term_stride, cw, t, nvalid);
+        }
+      } else {
+        if (whole || tail_valid)
+          ksb_chunk<XT, NB1>(acc, stg + r * kPitch + off0, stg + (r + 8) * kPitch + off1, xw,
+                             term_stride, cw, t);
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (++s == kStages) {
+        s = 0;
+        ph ^= 1u;
+      }
+      off0 = (off0 + kChunkBytes) & 15u;
+      off1 = (off1 + kChunkBytes) & 15u;
+      xw += x_chunk;
+      if (++cw_in_win == a.win) cw_in_win = 0;
     }
-    const int s = c % kStages;
-    if (!mbar_wait(&full[s], static_cast<uint32_t>(c / kStages) & 1u, a.budget) ||
-        *reinterpret_cast<volatile int*>(abort_flag)) {
-      ok = false;
-      break;
-    }
-    const int64_t b0 = static_cast<int64_t>(c) * kBlkPerChunk;
-    // byte offset of each row piece inside its first 16-byte granule
-    const uintptr_t base0 = reinterpret_cast<uintptr_t>(a.W) +
-                            static_cast<uintptr_t>((m0 + r) * a.rowbytes + b0 * kBlkB);
-    const uintptr_t base1 = base0 + static_cast<uintptr_t>(8 * a.rowbytes);
-    const uint32_t row0 = stages_addr + s * kStageBytes + r * kPitch + (base0 & 15u);
-    const uint32_t row1 = stages_addr + s * kStageBytes + (r + 8) * kPitch + (base1 & 15u);
-    const uint32_t xw = xs_addr + ((c % a.win) * a.B + bsel) * kXStride + t * 16;
+    if (!ok) break;
 
-    if constexpr (FMT == GQ_FMT_Q4_0) {
-      // this warp's 8 blocks of the chunk
-      const int jb0 = cw * 8;
-      const int nvalid = static_cast<int>(i64min(8, nblk_row - b0 - jb0));
-#pragma unroll 4
-      for (int j = 0; j < 8; ++j) {
-        if (j < nvalid) {
-          const uint32_t off = (jb0 + j) * kBlkB;
-          const float d0 = half_bits_to_float(lds16(row0 + off));
-          const float d1 = half_bits_to_float(lds16(row1 + off));
-          const uint32_t qa = lds32_even(row0 + off + 2 + 4 * t);
-          const uint32_t qb = lds32_even(row1 + off + 2 + 4 * t);
-          float cf[4] = {0.f, 0.f, 0.f, 0.f};
-          block_mma<XT>(cf, qa, qb, xw + (jb0 + j) * kXBlk, term_stride);
-          acc[0] = fmaf(d0, cf[0], acc[0]);
-          acc[1] = fmaf(d0, cf[1], acc[1]);
-          acc[2] = fmaf(d1, cf[2], acc[2]);
-          acc[3] = fmaf(d1, cf[3], acc[3]);
+    // reduce the consumer warps' partial sums (double-buffered by group
+    // parity, so one barrier per group suffices), then store
+    float* rb = red + (gi & 1) * kConsumers * 32 * 4;
+    reinterpret_cast<float4*>(rb)[cw * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    if (!group_sync()) { ok = false; break; }
+    if (cw == 0) {
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int w = 0; w < kConsumers; ++w) {
+        const float4 v = reinterpret_cast<const float4*>(rb)[w * 32 + lane];
+        s4[0] += v.x;
+        s4[1] += v.y;
+        s4[2] += v.z;
+        s4[3] += v.w;
+      }
+      const int64_t ra = m0 + r, rbw = m0 + r + 8;
+      if (NB1) {
+        if (t == 0) {
+          if (ra < a.M) store_elem(a.y, ra, s4[0], a.ytype);
+          if (rbw < a.M) store_elem(a.y, rbw, s4[2], a.ytype);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int col = 2 * t + i;
+          if (col < a.B) {
+            if (ra < a.M) store_elem(a.y, col * a.M + ra, s4[i], a.ytype);
+            if (rbw < a.M) store_elem(a.y, col * a.M + rbw, s4[2 + i], a.ytype);
+          }
         }
       }
-    } else {
-      // this warp's super-block of the chunk
-      if (b0 + cw < nblk_row) {
-        const uint32_t off = cw * kBlkB;
-        const float S0 = half_bits_to_float(lds16(row0 + off));
-        const float S1 = half_bits_to_float(lds16(row1 + off));
-        const uint32_t qs0a = lds32_even(row0 + off + 2), qs0b = lds32_even(row0 + off + 6);
-        const uint32_t qs1a = lds32_even(row1 + off + 2), qs1b = lds32_even(row1 + off + 6);
-        float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t qa = lds32_even(row0 + off + 10 + 16 * j + 4 * t);
-          const uint32_t qb = lds32_even(row1 + off + 10 + 16 * j + 4 * t);
-          float cf[4] = {0.f, 0.f, 0.f, 0.f};
-          block_mma<XT>(cf, qa, qb, xw + (cw * 8 + j) * kXBlk, term_stride);
-          const uint32_t w0 = (j < 4) ? qs0a : qs0b, w1 = (j < 4) ? qs1a : qs1b;
-          const float qj0 = static_cast<float>(static_cast<int8_t>((w0 >> (8 * (j & 3))) & 0xFFu));
-          const float qj1 = static_cast<float>(static_cast<int8_t>((w1 >> (8 * (j & 3))) & 0xFFu));
-          sacc[0] = fmaf(qj0, cf[0], sacc[0]);
-          sacc[1] = fmaf(qj0, cf[1], sacc[1]);
-          sacc[2] = fmaf(qj1, cf[2], sacc[2]);
-          sacc[3] = fmaf(qj1, cf[3], sacc[3]);
-        }
-        acc[0] = fmaf(S0, sacc[0], acc[0]);
-        acc[1] = fmaf(S0, sacc[1], acc[1]);
-        acc[2] = fmaf(S1, sacc[2], acc[2]);
-        acc[3] = fmaf(S1, sacc[3], acc[3]);
-      }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
   }
 
-  if (!ok) {
-    if (lane == 0) {
-      report(a.dev_status, GQ_DEV_TIMEOUT);
-      *reinterpret_cast<volatile int*>(abort_flag) = 1;
-    }
-    return;
-  }
-
-  // reduce the four consumer warps' partial sums, then store
-  float* my = red + (cw * 32 + lane) * 4;
-  my[0] = acc[0];
-  my[1] = acc[1];
-  my[2] = acc[2];
-  my[3] = acc[3];
-  if (!group_sync()) {
-    if (lane == 0) report(a.dev_status, GQ_DEV_TIMEOUT);
-    return;
-  }
-  if (cw == 0) {
-    float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int w = 0; w < kConsumers; ++w) {
-      const float* p = red + (w * 32 + lane) * 4;
-      s4[0] += p[0];
-      s4[1] += p[1];
-      s4[2] += p[2];
-      s4[3] += p[3];
-    }
-    const int64_t ra = m0 + r, rb = m0 + r + 8;
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int col = 2 * t + i;
-      if (col < a.B) {
-        if (ra < a.M) store_elem(a.y, col * a.M + ra, s4[i], a.ytype);
-        if (rb < a.M) store_elem(a.y, col * a.M + rb, s4[2 + i], a.ytype);
-      }
-    }
+  if (!ok && lane == 0) {
+    report(a.dev_status, GQ_DEV_TIMEOUT);
+    *reinterpret_cast<volatile int*>(abort_flag) = 1;
   }
 }
 
 size_t gemv_smem_bytes(int B, int terms, int win) {
   return static_cast<size_t>(kStages) * kStageBytes +
-         static_cast<size_t>(terms) * win * B * kXStride + kConsumers * 32 * 4 * sizeof(float) +
-         (2 * kStages + 1) * sizeof(uint64_t) + 16;
+         static_cast<size_t>(terms) * win * B * kXStride +
+         2 * kConsumers * 32 * 4 * sizeof(float) + (2 * kStages + 1) * sizeof(uint64_t) + 16;
 }
 
-template <int FMT, int XT>
-gq_status launch_gemv(const GemvArgs& a, cudaStream_t stream, bool pdl) {
+template <int FMT, int XT, bool NB1, bool ALIGNED>
+gq_status launch_gemv(GemvArgs a, cudaStream_t stream, bool pdl) {
   constexpr int kTerms = (XT == XT_F32) ? 3 : 1;
+  auto kern = gemv_kernel<FMT, XT, NB1, ALIGNED>;
   const size_t smem = gemv_smem_bytes(a.B, kTerms, a.win);
   static int configured_dev = -1;
-  static size_t configured = 0;
+  static size_t configured_smem = 0;
+  static size_t occ_smem = 0;
+  static int occupancy = 1;
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_dev != dev || configured < smem) {
-    const size_t want = static_cast<size_t>(kStages) * kStageBytes + kXSmemMax + 8192;
-    if (cudaFuncSetAttribute(gemv_kernel<FMT, XT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
+  if (configured_dev != dev || smem > configured_smem) {
+    // at least the common sizes, and always this launch's own requirement
+    const size_t want = smem > gemv_smem_bytes(1, kTerms, 1) + kXSmemMax
+                            ? smem
+                            : gemv_smem_bytes(1, kTerms, 1) + kXSmemMax;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(want)) != cudaSuccess)
       return GQ_ERR_CUDA;
     configured_dev = dev;
-    configured = want;
+    configured_smem = want;
+    occ_smem = 0;
   }
-  const int64_t grid = (a.M + kRows - 1) / kRows;
-  return launch(gemv_kernel<FMT, XT>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem,
-                stream, pdl, a);
+  if (occ_smem != smem) {
+    int per_sm = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) != cudaSuccess ||
+        per_sm < 1)
+      per_sm = 1;
+    occupancy = per_sm;
+    occ_smem = smem;
+  }
+  const int64_t slots = static_cast<int64_t>(sm_count()) * occupancy;
+  const int grid = static_cast<int>(a.ngroups < slots ? a.ngroups : slots);
+  return launch(kern, dim3(grid), dim3(kThreads), smem, stream, pdl, a);
+}
+
+template <int FMT, int XT>
+gq_status dispatch_gemv(const GemvArgs& a, cudaStream_t s, bool pdl) {
+  const bool nb1 = (a.B == 1);
+  const bool aligned = (FMT == GQ_FMT_Q4_0) && (a.rowbytes % 16 == 0) &&
+                       (reinterpret_cast<uintptr_t>(a.W) % 16 == 0);
+  if (nb1) {
+    return aligned ? launch_gemv<FMT, XT, true, true>(a, s, pdl)
+                   : launch_gemv<FMT, XT, true, false>(a, s, pdl);
+  }
+  return aligned ? launch_gemv<FMT, XT, false, true>(a, s, pdl)
+                 : launch_gemv<FMT, XT, false, false>(a, s, pdl);
 }
 
 template <int FMT>
@@ -495,6 +704,7 @@ gq_status gemv_entry(const void* W, int64_t M, int64_t K, const void* x, int xt,
   a.B = static_cast<int>(B);
   a.ytype = yt;
   a.nchunks = static_cast<int>((K + kChunkW - 1) / kChunkW);
+  a.ngroups = static_cast<int>((M + kRows - 1) / kRows);
   const int terms = (xt == GQ_F32) ? 3 : 1;
   int win = kXSmemMax / (terms * a.B * kXStride);
   if (win < 1) win = 1;
@@ -504,9 +714,9 @@ gq_status gemv_entry(const void* W, int64_t M, int64_t K, const void* x, int xt,
   const bool pdl = (flags & GQ_GEMV_PDL) != 0;
   cudaStream_t s = as_stream(stream);
   switch (xt) {
-    case GQ_F16: return launch_gemv<FMT, XT_F16>(a, s, pdl);
-    case GQ_BF16: return launch_gemv<FMT, XT_BF16>(a, s, pdl);
-    default: return launch_gemv<FMT, XT_F32>(a, s, pdl);
+    case GQ_F16: return dispatch_gemv<FMT, XT_F16>(a, s, pdl);
+    case GQ_BF16: return dispatch_gemv<FMT, XT_BF16>(a, s, pdl);
+    default: return dispatch_gemv<FMT, XT_F32>(a, s, pdl);
   }
 }
 
