@@ -31,6 +31,7 @@ EXPORTS = (
     "gq_quantize_q4_0", "gq_quantize_ksb",
     "gq_dequantize_q4_0", "gq_dequantize_ksb",
     "gq_gemv_q4_0", "gq_gemv_ksb",
+    "gq_gemm_workspace_bytes", "gq_gemm_q4_0", "gq_gemm_ksb",
 )
 
 _DTYPE_CODE = {torch.float32: GQ_F32, torch.float16: GQ_F16, torch.bfloat16: GQ_BF16}
@@ -68,6 +69,12 @@ def _load() -> ctypes.CDLL:
     for name in ("gq_gemv_q4_0", "gq_gemv_ksb"):
         f = getattr(L, name)
         f.argtypes = [vp, i64, i64, vp, c_int, i64, vp, c_int, c_uint, vp, vp]
+        f.restype = c_int
+    L.gq_gemm_workspace_bytes.argtypes = [c_int, i64, i64, i64]
+    L.gq_gemm_workspace_bytes.restype = ctypes.c_size_t
+    for name in ("gq_gemm_q4_0", "gq_gemm_ksb"):
+        f = getattr(L, name)
+        f.argtypes = [vp, i64, i64, vp, c_int, i64, vp, c_int, vp, ctypes.c_size_t, vp, vp]
         f.restype = c_int
     return L
 
@@ -183,3 +190,43 @@ def gq_gemv_ksb(W: torch.Tensor, M: int, K: int, x: torch.Tensor, y_dtype=torch.
                 dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """y[B, M] = W_hat[M, K] @ x[B, K]^T for super-block weights; B in 1..8."""
     return _gemv("gq_gemv_ksb", W, M, K, x, y_dtype, out, flags, dev_status, stream)
+
+
+def gq_gemm_workspace_bytes(fmt: int, M: int, K: int, B: int) -> int:
+    return int(lib.gq_gemm_workspace_bytes(int(fmt), int(M), int(K), int(B)))
+
+
+def _gemm(name: str, fmt: int, W: torch.Tensor, M: int, K: int, X: torch.Tensor, y_dtype, out,
+          workspace, dev_status, stream):
+    X2 = X if X.dim() == 2 else X.reshape(1, -1)
+    B = X2.shape[0]
+    if X2.shape[1] != K:
+        raise ValueError(f"X has {X2.shape[1]} columns, expected K={K}")
+    if X2.dtype not in _DTYPE_CODE or y_dtype not in _DTYPE_CODE:
+        raise TypeError("X must be bfloat16; Y float32, float16 or bfloat16")
+    if out is None:
+        out = torch.empty((B, M), dtype=y_dtype, device=X2.device)
+    need = gq_gemm_workspace_bytes(fmt, M, K, B)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X2.device)
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(getattr(lib, name)(_ptr(W), int(M), int(K), _ptr(X2), _DTYPE_CODE[X2.dtype], B,
+                              _ptr(out), _DTYPE_CODE[out.dtype], _ptr(workspace), ws_bytes,
+                              _ptr(dev_status), _stream(stream)), name)
+    return out
+
+
+def gq_gemm_q4_0(W: torch.Tensor, M: int, K: int, X: torch.Tensor, y_dtype=torch.float32,
+                 out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                 dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y[B, M] = W_hat[M, K] @ X[B, K]^T on the tensor cores (X bfloat16, B <= 256)."""
+    return _gemm("gq_gemm_q4_0", GQ_FMT_Q4_0, W, M, K, X, y_dtype, out, workspace, dev_status,
+                 stream)
+
+
+def gq_gemm_ksb(W: torch.Tensor, M: int, K: int, X: torch.Tensor, y_dtype=torch.float32,
+                out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y[B, M] = W_hat[M, K] @ X[B, K]^T for super-block weights on the tensor cores."""
+    return _gemm("gq_gemm_ksb", GQ_FMT_KSB, W, M, K, X, y_dtype, out, workspace, dev_status,
+                 stream)

@@ -1,0 +1,529 @@
+// gq_gemm.cu -- dequantize-fused batched product Y = W_hat * X on the
+// tcgen05 tensor cores, for batches large enough to be a dense contraction.
+//
+// Operation: Y[n][m] = sum_k W_hat[m][k] * X[n][k], with W_hat decoded from
+// Q4_0 blocks ("GGUF 量化内幕 第4章" 4.3: d * (code - 8)) or super-blocks
+// ("GGUF K-quants" 套娃: (S * q_j) * (code - 8)).  X is bf16, Y fp32/bf16/fp16.
+//
+// Exactness: a decoded weight has at most 14 significant bits, so it is the
+// exact sum of two bfloat16 numbers, hi = its top 8 significant bits and
+// lo = the rest.  Both tiles go through the tensor core against the same X
+// tile into one fp32 accumulator: every product is exact, only the fp32
+// accumulation rounds.
+//
+// Design (sm_100a, one 128-row tile of W per CTA, all of the batch as N):
+//  * warp 0 (producer): streams the tile's packed rows, 512 weights per row
+//    per stage, with one 1-D bulk copy per row (no multicast), and the X
+//    k-slices (64 x N bf16) with a 2-D TMA load in the 128-byte swizzle;
+//  * warps 2..5 (dequant, one thread per W row): decode each 64-weight
+//    k-step into the hi and lo bf16 tiles, written straight into the
+//    K-major 128-byte-swizzled UMMA layout, then fence the async proxy;
+//  * warp 1 (MMA): allocates the fp32 accumulator in tensor memory and one
+//    thread issues tcgen05.mma (M=128, N, K=16) for hi and lo per k16,
+//    releasing stages with tcgen05.commit;
+//  * warps 2..5 then read the accumulator with tcgen05.ld (each warp its
+//    32 TMEM lanes) and store Y.
+//  * Every wait is bounded; on expiry the kernel sets GQ_DEV_TIMEOUT, lets
+//    its own copies and MMAs land (bounded), frees TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gq.h"
+#include "gq_device.cuh"
+#include "gq_host.h"
+#include "gq_tc.cuh"
+
+namespace gq {
+namespace {
+
+constexpr int kBM = 128;                       // W rows per tile (UMMA M)
+constexpr int kBK = 64;                        // k per A/X stage (128-byte bf16 rows)
+constexpr int kWChunk = 512;                   // weights per W row per stage
+constexpr int kWPitch = 304;                   // >= 288 + 14, multiple of 16
+constexpr int kWStageBytes = kBM * kWPitch + 16;
+constexpr int kWStages = 2;
+constexpr int kAStages = 2;
+constexpr int kXStages = 2;
+constexpr int kATile = kBM * kBK * 2;          // one bf16 tile (hi or lo): 16 KB
+constexpr int kStepsPerChunk = kWChunk / kBK;  // 8
+constexpr int kDequantWarps = 4;
+constexpr int kThreads = 32 * (2 + kDequantWarps);
+
+template <int FMT>
+struct GFmt;
+template <>
+struct GFmt<GQ_FMT_Q4_0> {
+  static constexpr int kBlkW = 32, kBlkB = 18;
+};
+template <>
+struct GFmt<GQ_FMT_KSB> {
+  static constexpr int kBlkW = 256, kBlkB = 138;
+};
+
+struct GemmArgs {
+  const uint8_t* W;
+  int64_t M, K, rowbytes;
+  void* Y;
+  int* dev_status;
+  long long budget;
+  int B, N, ytype, nsteps, nchunks;
+  uint32_t tmem_cols;
+};
+
+struct Smem {
+  uint32_t a, x, w;  // byte offsets of the A, X and W rings
+  uint32_t x_stage;  // bytes per X stage
+};
+
+extern __shared__ __align__(1024) uint8_t gsm[];
+
+// Ring offsets inside dynamic shared memory, from a 1024-byte-aligned base
+// (the 128-byte swizzle atoms and the TMA destinations need that alignment).
+__device__ __forceinline__ Smem smem_layout(int N) {
+  Smem s;
+  const uint32_t base = smem_addr(gsm);
+  s.a = ((base + 1023u) & ~1023u) - base;
+  s.x = s.a + kAStages * 2 * kATile;
+  s.x_stage = static_cast<uint32_t>(N) * kBK * 2;
+  s.w = s.x + kXStages * s.x_stage;
+  return s;
+}
+
+__device__ __forceinline__ uint32_t g_ld32(uint32_t off) {
+  return *reinterpret_cast<const uint32_t*>(gsm + off);
+}
+__device__ __forceinline__ uint32_t g_ld16(uint32_t off) {
+  return *reinterpret_cast<const uint16_t*>(gsm + off);
+}
+__device__ __forceinline__ uint32_t g_ld32_even(uint32_t off) {
+  const uint32_t b = off & ~3u;
+  return __byte_perm(g_ld32(b), g_ld32(b + 4), (off & 2u) ? 0x5432u : 0x3210u);
+}
+
+// Exact split of a decoded weight w (<= 14 significant bits): hi keeps the
+// top bfloat16 bits, lo = w - hi is itself a bfloat16 number.
+__device__ __forceinline__ void split_pair(float w0, float w1, uint32_t& hi, uint32_t& lo) {
+  const uint32_t u0 = __float_as_uint(w0), u1 = __float_as_uint(w1);
+  const uint32_t h0 = u0 & 0xFFFF0000u, h1 = u1 & 0xFFFF0000u;
+  const float l0 = __fsub_rn(w0, __uint_as_float(h0));
+  const float l1 = __fsub_rn(w1, __uint_as_float(h1));
+  hi = __byte_perm(h0, h1, 0x7632u);
+  lo = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632u);
+}
+
+// Eight weights s * (code - 8) from eight nibbles (byte i of words wa|wb, low
+// or high nibble), as hi/lo bf16 16-byte chunks.
+__device__ __forceinline__ void decode8(uint32_t wa, uint32_t wb, int sh, float s, uint4& hi,
+                                        uint4& lo) {
+  float w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t word = (i < 4) ? wa : wb;
+    const uint32_t nib = (word >> (8 * (i & 3) + sh)) & 15u;
+    // (float)(nib - 8) exactly, via the 2^23 exponent bias
+    const float f = __fsub_rn(__uint_as_float(0x4B000000u | nib), 8388616.0f);
+    w[i] = __fmul_rn(s, f);
+  }
+  split_pair(w[0], w[1], hi.x, lo.x);
+  split_pair(w[2], w[3], hi.y, lo.y);
+  split_pair(w[4], w[5], hi.z, lo.z);
+  split_pair(w[6], w[7], hi.w, lo.w);
+}
+
+// Store chunk c (k = 8c .. 8c+7 of the 64-wide step) of row `row` into a
+// K-major 128-byte-swizzled bf16 tile.
+__device__ __forceinline__ void st_chunk(uint32_t tile, int row, int c, uint4 v) {
+  const uint32_t off = tile + (row >> 3) * 1024 + (row & 7) * 128 + ((c ^ (row & 7)) << 4);
+  *reinterpret_cast<uint4*>(gsm + off) = v;
+}
+
+// Decode one 32-weight block (scale s, 16 code bytes at `qs`) into chunks
+// c0 .. c0+3 of the hi and lo tiles.
+__device__ __forceinline__ void block_to_tiles(uint32_t qs, float s, uint32_t a_hi, uint32_t a_lo,
+                                               int row, int c0) {
+  const uint32_t q0 = g_ld32_even(qs), q1 = g_ld32_even(qs + 4);
+  const uint32_t q2 = g_ld32_even(qs + 8), q3 = g_ld32_even(qs + 12);
+  uint4 h, l;
+  decode8(q0, q1, 0, s, h, l);  // weights 0..7: low nibbles of qs[0..7]
+  st_chunk(a_hi, row, c0 + 0, h);
+  st_chunk(a_lo, row, c0 + 0, l);
+  decode8(q2, q3, 0, s, h, l);  // weights 8..15
+  st_chunk(a_hi, row, c0 + 1, h);
+  st_chunk(a_lo, row, c0 + 1, l);
+  decode8(q0, q1, 4, s, h, l);  // weights 16..23: high nibbles of qs[0..7]
+  st_chunk(a_hi, row, c0 + 2, h);
+  st_chunk(a_lo, row, c0 + 2, l);
+  decode8(q2, q3, 4, s, h, l);  // weights 24..31
+  st_chunk(a_hi, row, c0 + 3, h);
+  st_chunk(a_lo, row, c0 + 3, l);
+}
+
+__device__ __forceinline__ void zero_chunks(uint32_t a_hi, uint32_t a_lo, int row, int c0) {
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    st_chunk(a_hi, row, c0 + i, z);
+    st_chunk(a_lo, row, c0 + i, z);
+  }
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
+  constexpr int kBlkW = GFmt<FMT>::kBlkW, kBlkB = GFmt<FMT>::kBlkB;
+  constexpr int kChunkBytes = kWChunk / kBlkW * kBlkB;  // 288 or 276
+  const Smem L = smem_layout(a.N);
+  const uint32_t sbase = smem_addr(gsm);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gsm + L.w + kWStages * kWStageBytes);
+  uint64_t* w_full = bars;
+  uint64_t* w_empty = w_full + kWStages;
+  uint64_t* a_full = w_empty + kWStages;
+  uint64_t* a_empty = a_full + kAStages;
+  uint64_t* x_full = a_empty + kAStages;
+  uint64_t* x_empty = x_full + kXStages;
+  uint64_t* d_full = x_empty + kXStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(d_full + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kBM;
+  const int64_t nblk_row = a.K / kBlkW;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kWStages; ++i) {
+      mbar_init(&w_full[i], 1);
+      mbar_init(&w_empty[i], kDequantWarps);
+    }
+    for (int i = 0; i < kAStages; ++i) {
+      mbar_init(&a_full[i], kDequantWarps);
+      mbar_init(&a_empty[i], 1);
+    }
+    for (int i = 0; i < kXStages; ++i) {
+      mbar_init(&x_full[i], 1);
+      mbar_init(&x_empty[i], 1);
+    }
+    mbar_init(d_full, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, a.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+  auto aborted = [&]() { return *reinterpret_cast<volatile int*>(abort_flag) != 0; };
+  auto fail = [&]() {
+    report(a.dev_status, GQ_DEV_TIMEOUT);
+    *reinterpret_cast<volatile int*>(abort_flag) = 1;
+  };
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    // Issue order: W chunk c before the X step that first needs it.
+    int w_issued = 0, x_issued = 0;
+    bool ok = true;
+    for (int ks = 0; ks < a.nsteps && ok; ++ks) {
+      if (ks % kStepsPerChunk == 0) {
+        const int c = ks / kStepsPerChunk, s = c % kWStages;
+        if (!mbar_wait(&w_empty[s], ((c / kWStages) & 1u) ^ 1u, a.budget) || aborted()) {
+          ok = false;
+          break;
+        }
+        const int64_t b0 = static_cast<int64_t>(c) * (kWChunk / kBlkW);
+        const uint32_t nbytes = static_cast<uint32_t>(i64min(kWChunk / kBlkW, nblk_row - b0) * kBlkB);
+        uint32_t total = 0;
+        uintptr_t lo[4];
+        uint32_t len[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = lane + 32 * i;
+          len[i] = 0;
+          if (m0 + r < a.M) {
+            const uintptr_t src = reinterpret_cast<uintptr_t>(a.W) +
+                                  static_cast<uintptr_t>((m0 + r) * a.rowbytes + b0 * kBlkB);
+            lo[i] = src & ~static_cast<uintptr_t>(15);
+            len[i] = static_cast<uint32_t>(((src + nbytes + 15) & ~static_cast<uintptr_t>(15)) - lo[i]);
+          }
+          total += len[i];
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xFFFFFFFFu, total, o);
+        if (lane == 0) mbar_arrive_expect_tx(&w_full[s], total);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (len[i])
+            bulk_g2s(gsm + L.w + s * kWStageBytes + (lane + 32 * i) * kWPitch,
+                     reinterpret_cast<const void*>(lo[i]), len[i], &w_full[s], policy_evict_first());
+        w_issued = c + 1;
+      }
+      const int sx = ks % kXStages;
+      if (!mbar_wait(&x_empty[sx], ((ks / kXStages) & 1u) ^ 1u, a.budget) || aborted()) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&x_full[sx], L.x_stage);
+        tma_load_2d(gsm + L.x + sx * L.x_stage, &xmap, ks * kBK, 0, &x_full[sx]);
+      }
+      __syncwarp();
+      x_issued = ks + 1;
+    }
+    if (!ok && lane == 0) fail();
+    // let every issued copy land before shared memory is released
+    if (lane == 0) {
+      for (int c = max(0, w_issued - kWStages); c < w_issued; ++c)
+        if (!mbar_wait(&w_full[c % kWStages], (c / kWStages) & 1u, a.budget)) {
+          report(a.dev_status, GQ_DEV_TIMEOUT);
+          break;
+        }
+      for (int k = max(0, x_issued - kXStages); k < x_issued; ++k)
+        if (!mbar_wait(&x_full[k % kXStages], (k / kXStages) & 1u, a.budget)) {
+          report(a.dev_status, GQ_DEV_TIMEOUT);
+          break;
+        }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16(kBM, a.N);
+      bool ok = true;
+      for (int ks = 0; ks < a.nsteps; ++ks) {
+        const int sa = ks % kAStages, sx = ks % kXStages;
+        if (!mbar_wait(&a_full[sa], (ks / kAStages) & 1u, a.budget) ||
+            !mbar_wait(&x_full[sx], (ks / kXStages) & 1u, a.budget) || aborted()) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_hi = sbase + L.a + sa * 2 * kATile, a_lo = a_hi + kATile;
+        const uint32_t xs = sbase + L.x + sx * L.x_stage;
+#pragma unroll
+        for (int k16 = 0; k16 < kBK / 16; ++k16) {
+          const uint64_t xd = umma_desc_sw128(xs + 32 * k16);
+          umma_bf16(tmem_d, umma_desc_sw128(a_hi + 32 * k16), xd, idesc, (ks | k16) != 0);
+          umma_bf16(tmem_d, umma_desc_sw128(a_lo + 32 * k16), xd, idesc, 1u);
+        }
+        umma_commit(&a_empty[sa]);
+        umma_commit(&x_empty[sx]);
+      }
+      if (!ok) fail();
+      // d_full completes once every MMA issued above has finished (also on
+      // the abort path, so that TMEM and shared memory are quiet before exit)
+      umma_commit(d_full);
+    }
+    __syncwarp();
+  } else {
+    // ----------------------------------------------------------- dequant
+    const int row = (warp & 3) * 32 + lane;  // TMEM lane quarter = warp % 4
+    const bool row_ok = m0 + row < a.M;
+    const uintptr_t row_addr =
+        reinterpret_cast<uintptr_t>(a.W) + static_cast<uintptr_t>((m0 + (row_ok ? row : 0)) * a.rowbytes);
+    bool ok = true;
+    for (int ks = 0; ks < a.nsteps && ok; ++ks) {
+      const int c = ks / kStepsPerChunk, j = ks % kStepsPerChunk, sw = c % kWStages;
+      if (j == 0 && (!mbar_wait(&w_full[sw], (c / kWStages) & 1u, a.budget) || aborted())) {
+        ok = false;
+        break;
+      }
+      const int sa = ks % kAStages;
+      if (!mbar_wait(&a_empty[sa], ((ks / kAStages) & 1u) ^ 1u, a.budget) || aborted()) {
+        ok = false;
+        break;
+      }
+      const uint32_t a_hi = L.a + sa * 2 * kATile, a_lo = a_hi + kATile;
+      // this row's piece of the chunk, from its offset inside the first granule
+      const uint32_t slot = L.w + sw * kWStageBytes + row * kWPitch +
+                            static_cast<uint32_t>((row_addr + static_cast<uintptr_t>(c) * kChunkBytes) & 15u);
+      const int64_t blk0 = static_cast<int64_t>(c) * (kWChunk / kBlkW);  // first block of the chunk
+      if constexpr (FMT == GQ_FMT_Q4_0) {
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const int jb = 2 * j + bb;  // block within the chunk
+          if (blk0 + jb < nblk_row) {
+            const uint32_t o = slot + jb * 18;
+            block_to_tiles(o + 2, half_bits_to_float(g_ld16(o)), a_hi, a_lo, row, 4 * bb);
+          } else {
+            zero_chunks(a_hi, a_lo, row, 4 * bb);
+          }
+        }
+      } else {
+        const int sb = j >> 2;  // super-block within the chunk
+        const uint32_t o = slot + sb * 138;
+        if (blk0 + sb < nblk_row) {
+          const float S = half_bits_to_float(g_ld16(o));
+#pragma unroll
+          for (int bb = 0; bb < 2; ++bb) {
+            const int sub = 2 * (j & 3) + bb;
+            const uint32_t qw = g_ld16(o + 2 + (sub & ~1));
+            const int qj = static_cast<int8_t>((qw >> (8 * (sub & 1))) & 0xFFu);
+            block_to_tiles(o + 10 + 16 * sub, __fmul_rn(S, static_cast<float>(qj)), a_hi, a_lo, row,
+                           4 * bb);
+          }
+        } else {
+          zero_chunks(a_hi, a_lo, row, 0);
+          zero_chunks(a_hi, a_lo, row, 4);
+        }
+      }
+      fence_proxy_async_smem();  // generic writes -> visible to the tensor core
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&a_full[sa]);
+        if (j == kStepsPerChunk - 1 || ks == a.nsteps - 1) mbar_arrive(&w_empty[sw]);
+      }
+    }
+    if (!ok && lane == 0) fail();
+
+    // ---------------------------------------------------------- epilogue
+    if (mbar_wait(d_full, 0, a.budget)) {
+      tc_fence_after();
+      if (__all_sync(0xFFFFFFFFu, ok && !aborted())) {  // tcgen05.ld is warp-collective
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        for (int n0 = 0; n0 < a.N; n0 += 16) {
+          uint32_t v[16];
+          tmem_ld16(tmem_d + lane_base + n0, v);
+          tmem_wait_ld();
+          if (row_ok) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (n0 + i < a.B) store_elem(a.Y, (n0 + i) * a.M + m0 + row, __uint_as_float(v[i]), a.ytype);
+          }
+        }
+      }
+    } else if (lane == 0) {
+      report(a.dev_status, GQ_DEV_TIMEOUT);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_d, a.tmem_cols);
+  }
+}
+
+size_t gemm_smem_bytes(int N) {
+  return static_cast<size_t>(kAStages) * 2 * kATile + static_cast<size_t>(kXStages) * N * kBK * 2 +
+         static_cast<size_t>(kWStages) * kWStageBytes + 16 * sizeof(uint64_t) + 1024;
+}
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+  static EncodeTiled fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(p);
+  }
+  return fn;
+}
+
+template <int FMT>
+gq_status gemm_entry(const void* W, int64_t M, int64_t K, const void* X, int xt, int64_t B, void* Y,
+                     int yt, void* workspace, size_t ws_bytes, int* dev_status, void* stream) {
+  constexpr int kBlkW = GFmt<FMT>::kBlkW, kBlkB = GFmt<FMT>::kBlkB;
+  (void)workspace;
+  (void)ws_bytes;
+  if (M < 0 || K < 0 || B < 0) return GQ_ERR_INVALID_ARG;
+  if (xt != GQ_BF16 || !valid_act_dtype(yt)) return GQ_ERR_DTYPE;
+  if (K % kBlkW) return GQ_ERR_SHAPE;
+  if (B > 256 || M > 0x7FFFFFFFLL || K > (1LL << 24)) return GQ_ERR_SHAPE;
+  if (M == 0 || B == 0) return GQ_OK;
+  if (!Y) return GQ_ERR_INVALID_ARG;
+  if (misaligned16(Y)) return GQ_ERR_ALIGNMENT;
+  if (K == 0) {
+    return cudaMemsetAsync(Y, 0, static_cast<size_t>(B * M * dtype_size(yt)), as_stream(stream)) ==
+                   cudaSuccess
+               ? GQ_OK
+               : GQ_ERR_CUDA;
+  }
+  if (!W || !X) return GQ_ERR_INVALID_ARG;
+  if (misaligned16(W) || misaligned16(X)) return GQ_ERR_ALIGNMENT;
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return GQ_ERR_ALIGNMENT;
+
+  EncodeTiled enc = encode_fn();
+  if (!enc) return GQ_ERR_CUDA;
+  const int N = static_cast<int>((B + 15) / 16 * 16);
+  CUtensorMap xmap;
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(B)};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(N)};
+  const cuuint32_t estride[2] = {1, 1};
+  if (enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(X), gdim, gstride, box,
+          estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return GQ_ERR_CUDA;
+
+  GemmArgs a;
+  a.W = static_cast<const uint8_t*>(W);
+  a.M = M;
+  a.K = K;
+  a.rowbytes = K / kBlkW * kBlkB;
+  a.Y = Y;
+  a.dev_status = dev_status;
+  a.budget = kWaitBudget;
+  a.B = static_cast<int>(B);
+  a.N = N;
+  a.ytype = yt;
+  a.nsteps = static_cast<int>((K + kBK - 1) / kBK);
+  a.nchunks = static_cast<int>((K + kWChunk - 1) / kWChunk);
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(N)) cols <<= 1;
+  a.tmem_cols = cols;
+
+  const size_t smem = gemm_smem_bytes(N);
+  static int configured_dev = -1;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
+  if (configured_dev != dev) {
+    if (cudaFuncSetAttribute(gemm_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(gemm_smem_bytes(256))) != cudaSuccess)
+      return GQ_ERR_CUDA;
+    configured_dev = dev;
+  }
+  const int64_t grid = (M + kBM - 1) / kBM;
+  return launch(gemm_kernel<FMT>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem,
+                as_stream(stream), false, xmap, a);
+}
+
+}  // namespace
+}  // namespace gq
+
+extern "C" {
+
+GQ_API size_t gq_gemm_workspace_bytes(int fmt, int64_t M, int64_t K, int64_t B) {
+  (void)fmt;
+  (void)M;
+  (void)K;
+  (void)B;
+  return 0;
+}
+
+GQ_API gq_status gq_gemm_q4_0(const void* W, int64_t M, int64_t K, const void* X, int x_dtype,
+                              int64_t B, void* Y, int y_dtype, void* workspace, size_t ws_bytes,
+                              int* dev_status, void* stream) {
+  return gq::gemm_entry<GQ_FMT_Q4_0>(W, M, K, X, x_dtype, B, Y, y_dtype, workspace, ws_bytes,
+                                     dev_status, stream);
+}
+
+GQ_API gq_status gq_gemm_ksb(const void* W, int64_t M, int64_t K, const void* X, int x_dtype,
+                             int64_t B, void* Y, int y_dtype, void* workspace, size_t ws_bytes,
+                             int* dev_status, void* stream) {
+  return gq::gemm_entry<GQ_FMT_KSB>(W, M, K, X, x_dtype, B, Y, y_dtype, workspace, ws_bytes,
+                                    dev_status, stream);
+}
+
+}  // extern "C"

@@ -153,6 +153,30 @@ GQ_API gq_status gq_gemv_ksb(const void* W, int64_t M, int64_t K,
                              void* y, int y_dtype, unsigned flags,
                              int* dev_status, void* stream);
 
+/* Dequantize-fused batched product for batches that make a dense
+ * contraction: Y = W_hat * X^T on the tcgen05 tensor cores (the matrix
+ * multiply that consumes decoded blocks, Q4_0 chapter 4.3).
+ *   W: M x K packed as for gq_gemv_*.  K % 32 == 0 (Q4_0) / K % 256 == 0 (KSB).
+ *   X: [B][K] bfloat16 (x_dtype must be GQ_BF16), row-major, 16-byte aligned.
+ *   Y: [B][M] of y_dtype (GQ_F32, GQ_F16 or GQ_BF16), row-major.
+ *   B: 1..256 (0 launches nothing).
+ * Arithmetic: each decoded weight (at most 14 significant bits) is split
+ * exactly into two bfloat16 parts, both multiplied by X on the tensor core
+ * into one fp32 accumulator, so every product is exact and only the fp32
+ * accumulation rounds.
+ * workspace / ws_bytes: caller-owned scratch of at least
+ * gq_gemm_workspace_bytes(...) bytes (may be NULL when that is 0).
+ * dev_status: optional, receives GQ_DEV_TIMEOUT if a pipeline wait gives up. */
+GQ_API size_t gq_gemm_workspace_bytes(int fmt, int64_t M, int64_t K, int64_t B);
+GQ_API gq_status gq_gemm_q4_0(const void* W, int64_t M, int64_t K,
+                              const void* X, int x_dtype, int64_t B,
+                              void* Y, int y_dtype, void* workspace, size_t ws_bytes,
+                              int* dev_status, void* stream);
+GQ_API gq_status gq_gemm_ksb(const void* W, int64_t M, int64_t K,
+                             const void* X, int x_dtype, int64_t B,
+                             void* Y, int y_dtype, void* workspace, size_t ws_bytes,
+                             int* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

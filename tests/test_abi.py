@@ -112,3 +112,30 @@ def test_binding_refuses_host_tensors():
     import torch
     with pytest.raises(ValueError):
         gq.gq_quantize_q4_0(torch.zeros(64))
+
+
+@pytest.mark.parametrize("name,block", [("gq_gemm_q4_0", 32), ("gq_gemm_ksb", 256)])
+def test_gemm_validation(name, block):
+    f = getattr(gq.lib, name)
+    K = 4 * block
+    ok = dict(W=A, M=128, K=K, X=A, xt=2, B=16, Y=A, yt=0, ws=None, wsb=0, st=None, s=None)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["W"], a["M"], a["K"], a["X"], a["xt"], a["B"], a["Y"], a["yt"], a["ws"],
+                 a["wsb"], a["st"], a["s"])
+
+    assert call(M=-1) == INVALID
+    assert call(B=-2) == INVALID
+    assert call(xt=1) == DTYPE          # X must be bfloat16
+    assert call(yt=5) == DTYPE
+    assert call(K=K + 16) == SHAPE
+    assert call(B=257) == SHAPE
+    assert call(M=0) == GQ_OK and call(B=0) == GQ_OK
+    assert call(Y=None) == INVALID
+    assert call(W=None) == INVALID
+    assert call(X=None) == INVALID
+    assert call(W=A + 2) == ALIGN
+    assert call(X=A + 8) == ALIGN
+    assert call(st=A + 1) == ALIGN
+    assert gq.gq_gemm_workspace_bytes(0, 11008, 4096, 256) >= 0
