@@ -386,6 +386,141 @@ def run_reference(args, rank, ws):
     }
 
 
+# ------------------------------------------------------------------ suite
+def _timed(fn, reps, warmup=3):
+    """Device ms per call of fn(), CUDA events on the current stream."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def _graph_ms_per_launch(fn, launches, reps):
+    g = capture(fn)
+    ms = _timed(g.replay, reps)
+    del g
+    return ms / launches
+
+
+def run_suite(path):
+    """Every row of the hot path on its own workload; one JSON line per row."""
+    import torch
+    import bit_gemv_q4_b200 as gq
+    import synth
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peak, peak_src = measured_peaks()
+    out = open(path, "w")
+
+    def emit(d):
+        out.write(json.dumps(d) + "\n")
+        out.flush()
+        print("suite:", json.dumps(d), file=sys.stderr, flush=True)
+
+    def quant(fmt, w):
+        return (gq.gq_quantize_q4_0 if fmt == "q4_0" else gq.gq_quantize_ksb)(w.view(-1))
+
+    # --- single GEMVs (decode shapes), cold weights, graph + PDL
+    for fmt, M, K, B, xdt, ydt, name in (
+            ("q4_0", 256, 1024, 1, torch.float32, torch.float32, "tiny 256x1024 fp32"),
+            ("q4_0", 4096, 4096, 1, torch.float16, torch.float16, "decode 4096x4096"),
+            ("ksb", 11008, 4096, 1, torch.float16, torch.float16, "MLP 11008x4096 ksb B=1"),
+            ("ksb", 11008, 4096, 8, torch.float16, torch.float16, "MLP 11008x4096 ksb B=8"),
+            ("q4_0", 11008, 4096, 8, torch.float16, torch.float16, "MLP 11008x4096 q4_0 B=8")):
+        w = synth.gaussian_weights(M, K, seed=7, device=dev)
+        q = quant(fmt, w)
+        del w
+        nb = q.numel()
+        copies = max(4, int(512e6 // nb))
+        Wc = torch.empty((copies, nb), dtype=torch.uint8, device=dev)
+        Wc.copy_(q.view(1, nb).expand(copies, nb))
+        x = synth.activations(B, K, seed=8, dtype=xdt, device=dev)
+        y = torch.empty((B, M), dtype=ydt, device=dev)
+        f = gq.gq_gemv_q4_0 if fmt == "q4_0" else gq.gq_gemv_ksb
+        ms = _graph_ms_per_launch(
+            lambda: [f(Wc[i], M, K, x, y_dtype=ydt, out=y, flags=gq.GQ_GEMV_PDL) for i in range(copies)],
+            copies, 20)
+        emit({"row": "gemv", "workload": name, "format": fmt, "M": M, "K": K, "B": B,
+              "us": round(ms * 1e3, 3), "weight_gbs": round(nb / (ms * 1e-3) / 1e9, 1),
+              "frac_of_peak": round(nb / (ms * 1e-3) / 1e9 / peak, 4),
+              "gflops": round(2 * M * K * B / (ms * 1e-3) / 1e9, 1)})
+        del Wc
+
+    # --- whole-model weight stream: 32 layers x (4 x 4096^2 + 3 x 11008x4096)
+    for fmt in ("q4_0", "ksb"):
+        shapes = []
+        for layer in range(32):
+            shapes += [(4096, 4096)] * 4 + [(11008, 4096)] * 3
+        mats, total = [], 0
+        for i, (M, K) in enumerate(shapes):
+            w = synth.gaussian_weights(M, K, seed=30000 + i, device=dev)
+            mats.append((quant(fmt, w), M, K))
+            total += mats[-1][0].numel()
+            del w
+        x = synth.activations(1, 4096, seed=9, dtype=torch.float16, device=dev)
+        ys = {M: torch.empty((1, M), dtype=torch.float16, device=dev) for M in (4096, 11008)}
+        f = gq.gq_gemv_q4_0 if fmt == "q4_0" else gq.gq_gemv_ksb
+        ms = _graph_ms_per_launch(
+            lambda: [f(qm, M, K, x, out=ys[M], flags=gq.GQ_GEMV_PDL) for qm, M, K in mats], 1, 5)
+        emit({"row": "model_stream", "workload": "32 layers x (4 x 4096x4096 + 3 x 11008x4096), "
+              "224 batch-1 GEMVs, one CUDA graph", "format": fmt, "weight_bytes": total,
+              "ms": round(ms, 3), "weight_gbs": round(total / (ms * 1e-3) / 1e9, 1),
+              "frac_of_peak": round(total / (ms * 1e-3) / 1e9 / peak, 4),
+              "matrices_per_s": round(224 / (ms * 1e-3), 1)})
+        del mats
+        torch.cuda.empty_cache()
+
+    # --- tensor-core dequant-GEMM, W 11008x4096, X bf16 [B, 4096]
+    M, K = 11008, 4096
+    for fmt in ("q4_0", "ksb"):
+        w = synth.gaussian_weights(M, K, seed=11, device=dev)
+        q = quant(fmt, w)
+        del w
+        nb = q.numel()
+        copies = 6
+        Wc = torch.empty((copies, nb), dtype=torch.uint8, device=dev)
+        Wc.copy_(q.view(1, nb).expand(copies, nb))
+        f = gq.gq_gemm_q4_0 if fmt == "q4_0" else gq.gq_gemm_ksb
+        for B in (16, 64, 256):
+            X = synth.activations(B, K, seed=12, dtype=torch.bfloat16, device=dev)
+            Y = torch.empty((B, M), dtype=torch.float32, device=dev)
+            ms = _graph_ms_per_launch(lambda: [f(Wc[i], M, K, X, out=Y) for i in range(copies)],
+                                      copies, 10)
+            tf = 2.0 * M * K * B / (ms * 1e-3) / 1e12
+            emit({"row": "gemm", "workload": f"W {M}x{K} x X bf16 [{B},{K}], Y fp32",
+                  "format": fmt, "B": B, "us": round(ms * 1e3, 2), "tflops": round(tf, 1),
+                  "weight_gbs": round(nb / (ms * 1e-3) / 1e9, 1),
+                  "frac_of_bf16_peak": round(tf / 1615.2, 4),
+                  "note": "useful flops 2*M*K*B; the exact hi/lo split issues twice that"})
+        del Wc
+
+    # --- quantize and dequantize 1e9 weights ~ N(0, 0.02^2)
+    n = 1_000_000_000
+    w = synth.gaussian_weights(n // 8000, 8000, seed=4, frac=0.0, device=dev).view(-1)
+    for fmt, nbytes in (("q4_0", n // 32 * 18), ("ksb", n // 256 * 138)):
+        q = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        fq = gq.gq_quantize_q4_0 if fmt == "q4_0" else gq.gq_quantize_ksb
+        ms = _timed(lambda: fq(w, out=q), 5)
+        emit({"row": "quantize", "workload": "1e9 fp32 weights", "format": fmt,
+              "ms": round(ms, 3), "gweights_per_s": round(n / (ms * 1e-3) / 1e9, 2),
+              "gbs": round((4 * n + nbytes) / (ms * 1e-3) / 1e9, 1),
+              "frac_of_peak": round((4 * n + nbytes) / (ms * 1e-3) / 1e9 / peak, 4)})
+        fd = gq.gq_dequantize_q4_0 if fmt == "q4_0" else gq.gq_dequantize_ksb
+        ms = _timed(lambda: fd(q, n, out=w), 5)
+        emit({"row": "dequantize", "workload": "1e9 weights to fp32", "format": fmt,
+              "ms": round(ms, 3), "gweights_per_s": round(n / (ms * 1e-3) / 1e9, 2),
+              "gbs": round((4 * n + nbytes) / (ms * 1e-3) / 1e9, 1),
+              "frac_of_peak": round((4 * n + nbytes) / (ms * 1e-3) / 1e9 / peak, 4)})
+        del q
+    out.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -397,6 +532,8 @@ def main():
                     help="bounded sample of oracle work for cpu_baseline")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu DRAM bytes per launch of the GEMV kernel, if measured")
+    ap.add_argument("--suite", default=None,
+                    help="also measure every hot-path row; JSON lines written to this file")
     args = ap.parse_args()
 
     rank, ws, local = dist_setup()
@@ -409,6 +546,8 @@ def main():
                 v, cores, desc = OracleSample().run(args.cpu_seconds)
                 res["cpu_baseline"] = {"value": round(v, 3), "unit": "GB/s", "cores": cores,
                                        "kind": "oracle", "sample": desc}
+            if args.suite and rank == 0:
+                run_suite(args.suite)
         if rank == 0 and res is not None:
             print(json.dumps(res), flush=True)
     finally:
