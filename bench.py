@@ -35,6 +35,29 @@ METRIC = "Q4 GEMV streamed-weight GB/s and % of HBM peak (4096x11008, batch 1)"
 CASES = [("q4_0", 4096, 11008), ("q4_0", 11008, 4096), ("ksb", 4096, 11008), ("ksb", 11008, 4096)]
 FALLBACK_HBM_GBS = 6650.0
 
+# DRAM bytes per GEMV launch (mean over the four cases) from one ncu capture
+# (profiles/gemv_q4_0_4096x11008.md).  Reported only while the GEMV sources
+# hash to what was profiled; any change to the kernel makes it null.
+GEMV_TRAFFIC = {
+    "bytes": 25407744,
+    "sources": {
+        "bit_gemv_q4_b200/csrc/gq_gemv.cu": "c19aaf85ea5b879f2aaa30d2c6800b507f4e560801bb17aa0357e490d98e7537",
+        "bit_gemv_q4_b200/csrc/gq_device.cuh": "a2e2779ecb02fd76d9cd3c26065670d43d3cf6839efcb7fd46da6bc987ddcffd",
+    },
+}
+
+
+def gemv_traffic():
+    import hashlib
+    for rel, digest in GEMV_TRAFFIC["sources"].items():
+        try:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest() != digest:
+                    return None
+        except OSError:
+            return None
+    return GEMV_TRAFFIC["bytes"]
+
 
 def packed_bytes(fmt, M, K):
     return M * (K // 32 * 18 if fmt == "q4_0" else K // 256 * 138)
@@ -307,7 +330,7 @@ def run_ours(args, rank, ws, local):
         "frac_of_peak": round(gbs / ws / peak, 4),
         "roofline": {"bound": "hbm", "achieved": round(per_gpu_algo_gbs, 1), "peak": peak,
                      "peak_source": f"{peak_src} hbm_gbs", "unit": "GB/s",
-                     "frac": round(per_gpu_algo_gbs / peak, 4), "traffic": args.traffic,
+                     "frac": round(per_gpu_algo_gbs / peak, 4), "traffic": gemv_traffic(),
                      "kernel": "gemv_kernel (all four cases)"},
         "cases": cases,
         "no_pdl_gbs": round(nopdl_gbs, 1),
@@ -521,6 +544,38 @@ def run_suite(path):
     out.close()
 
 
+def run_single(spec, launches, batch, flags):
+    """A few launches of one product on distinct copies of one matrix (for
+    profilers): spec = "gemv:q4_0:4096:11008" or "gemm:ksb:11008:4096"."""
+    import torch
+    import bit_gemv_q4_b200 as gq
+    import synth
+    kind, fmt, M, K = spec.split(":")
+    M, K = int(M), int(K)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = synth.gaussian_weights(M, K, seed=1, device=dev)
+    q = (gq.gq_quantize_q4_0 if fmt == "q4_0" else gq.gq_quantize_ksb)(w.view(-1))
+    del w
+    nb = q.numel()
+    copies = 6
+    Wc = torch.empty((copies, nb), dtype=torch.uint8, device=dev)
+    Wc.copy_(q.view(1, nb).expand(copies, nb))
+    if kind == "gemv":
+        x = synth.activations(batch, K, seed=2, dtype=torch.float16, device=dev)
+        f = gq.gq_gemv_q4_0 if fmt == "q4_0" else gq.gq_gemv_ksb
+        y = torch.empty((batch, M), dtype=torch.float16, device=dev)
+        run = lambda i: f(Wc[i % copies], M, K, x, out=y, flags=flags)
+    else:
+        x = synth.activations(batch, K, seed=2, dtype=torch.bfloat16, device=dev)
+        f = gq.gq_gemm_q4_0 if fmt == "q4_0" else gq.gq_gemm_ksb
+        y = torch.empty((batch, M), dtype=torch.float32, device=dev)
+        run = lambda i: f(Wc[i % copies], M, K, x, out=y)
+    for i in range(launches):
+        run(i)
+    torch.cuda.synchronize()
+    print(json.dumps({"single": spec, "batch": batch, "launches": launches, "bytes": nb}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -530,11 +585,17 @@ def main():
     ap.add_argument("--copies", type=int, default=16)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="bounded sample of oracle work for cpu_baseline")
-    ap.add_argument("--traffic", type=float, default=None,
-                    help="ncu DRAM bytes per launch of the GEMV kernel, if measured")
     ap.add_argument("--suite", default=None,
                     help="also measure every hot-path row; JSON lines written to this file")
+    ap.add_argument("--single", default=None,
+                    help="profiling aid: launch one product a few times, e.g. gemv:q4_0:4096:11008")
+    ap.add_argument("--launches", type=int, default=4)
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--flags", type=int, default=0)
     args = ap.parse_args()
+    if args.single:
+        run_single(args.single, args.launches, args.batch, args.flags)
+        return
 
     rank, ws, local = dist_setup()
     try:

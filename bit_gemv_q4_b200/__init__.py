@@ -4,7 +4,7 @@ Every function below passes device pointers, sizes and the current CUDA stream
 to the C entry point of the same name and raises ``GQError`` on a non-OK
 status.  All arithmetic happens in the CUDA kernels of libgq.so; there is no
 Python or CPU fallback, and importing this package fails if the library has
-not been built (``python -m bit_gemv_q4_b200.build``).
+not been built (``python bit_gemv_q4_b200/build.py``).
 
 PyTorch is used only to allocate device memory and to name the stream.
 """
@@ -32,6 +32,7 @@ EXPORTS = (
     "gq_dequantize_q4_0", "gq_dequantize_ksb",
     "gq_gemv_q4_0", "gq_gemv_ksb",
     "gq_gemm_workspace_bytes", "gq_gemm_q4_0", "gq_gemm_ksb",
+    "gq_selftest_gemv_timeout",
 )
 
 _DTYPE_CODE = {torch.float32: GQ_F32, torch.float16: GQ_F16, torch.bfloat16: GQ_BF16}
@@ -46,7 +47,7 @@ class GQError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"libgq.so not found at {LIB_PATH}; build it with `python -m bit_gemv_q4_b200.build`")
+            f"libgq.so not found at {LIB_PATH}; build it with `python bit_gemv_q4_b200/build.py`")
     L = ctypes.CDLL(LIB_PATH)
     i64, vp, c_int, c_uint = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_uint
     L.gq_abi_version.restype = c_int
@@ -76,6 +77,8 @@ def _load() -> ctypes.CDLL:
         f = getattr(L, name)
         f.argtypes = [vp, i64, i64, vp, c_int, i64, vp, c_int, vp, ctypes.c_size_t, vp, vp]
         f.restype = c_int
+    L.gq_selftest_gemv_timeout.argtypes = [vp, i64, i64, vp, vp, vp, vp]
+    L.gq_selftest_gemv_timeout.restype = c_int
     return L
 
 
@@ -230,3 +233,12 @@ def gq_gemm_ksb(W: torch.Tensor, M: int, K: int, X: torch.Tensor, y_dtype=torch.
     """Y[B, M] = W_hat[M, K] @ X[B, K]^T for super-block weights on the tensor cores."""
     return _gemm("gq_gemm_ksb", GQ_FMT_KSB, W, M, K, X, y_dtype, out, workspace, dev_status,
                  stream)
+
+
+def gq_selftest_gemv_timeout(W: torch.Tensor, M: int, K: int, x: torch.Tensor, y: torch.Tensor,
+                             dev_status: torch.Tensor, stream=None) -> None:
+    """Run the GEMV with a first stage that never fills; the bounded wait must
+    report GQ_DEV_TIMEOUT in dev_status (see include/gq.h)."""
+    _check(lib.gq_selftest_gemv_timeout(_ptr(W), int(M), int(K), _ptr(x), _ptr(y),
+                                        _ptr(dev_status), _stream(stream)),
+           "gq_selftest_gemv_timeout")

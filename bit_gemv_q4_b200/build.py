@@ -1,6 +1,8 @@
 """Build libgq.so (the C-ABI CUDA library) in-tree with nvcc for sm_100a.
 
-    python -m bit_gemv_q4_b200.build [--force] [--ptxas-v]
+    python bit_gemv_q4_b200/build.py [--force] [--ptxas-v]
+
+(Run it by path: importing the package loads the library this file builds.)
 
 The library is self-contained (static CUDA runtime) and exports only the
 ``gq_*`` entry points declared in include/gq.h.

@@ -45,11 +45,12 @@ constexpr int kWChunk = 512;                   // weights per W row per stage
 constexpr int kWPitch = 304;                   // >= 288 + 14, multiple of 16
 constexpr int kWStageBytes = kBM * kWPitch + 16;
 constexpr int kWStages = 2;
-constexpr int kAStages = 2;
-constexpr int kXStages = 2;
+constexpr int kAStagesMax = 3;                 // decoded hi/lo tile pairs
+constexpr int kXStagesMax = 8;                 // activation k-slices
+constexpr int kSmemBudget = 227 * 1024;
 constexpr int kATile = kBM * kBK * 2;          // one bf16 tile (hi or lo): 16 KB
 constexpr int kStepsPerChunk = kWChunk / kBK;  // 8
-constexpr int kDequantWarps = 4;
+constexpr int kDequantWarps = 8;   // two per scheduler; each thread decodes one block per k-step
 constexpr int kThreads = 32 * (2 + kDequantWarps);
 
 template <int FMT>
@@ -70,6 +71,7 @@ struct GemmArgs {
   int* dev_status;
   long long budget;
   int B, N, ytype, nsteps, nchunks;
+  int astages, xstages;  // ring depths chosen from the shared-memory budget
   uint32_t tmem_cols;
 };
 
@@ -82,13 +84,13 @@ extern __shared__ __align__(1024) uint8_t gsm[];
 
 // Ring offsets inside dynamic shared memory, from a 1024-byte-aligned base
 // (the 128-byte swizzle atoms and the TMA destinations need that alignment).
-__device__ __forceinline__ Smem smem_layout(int N) {
+__device__ __forceinline__ Smem smem_layout(int N, int astages, int xstages) {
   Smem s;
   const uint32_t base = smem_addr(gsm);
   s.a = ((base + 1023u) & ~1023u) - base;
-  s.x = s.a + kAStages * 2 * kATile;
+  s.x = s.a + astages * 2 * kATile;
   s.x_stage = static_cast<uint32_t>(N) * kBK * 2;
-  s.w = s.x + kXStages * s.x_stage;
+  s.w = s.x + xstages * s.x_stage;
   return s;
 }
 
@@ -98,39 +100,44 @@ __device__ __forceinline__ uint32_t g_ld32(uint32_t off) {
 __device__ __forceinline__ uint32_t g_ld16(uint32_t off) {
   return *reinterpret_cast<const uint16_t*>(gsm + off);
 }
-__device__ __forceinline__ uint32_t g_ld32_even(uint32_t off) {
-  const uint32_t b = off & ~3u;
-  return __byte_perm(g_ld32(b), g_ld32(b + 4), (off & 2u) ? 0x5432u : 0x3210u);
-}
 
-// Exact split of a decoded weight w (<= 14 significant bits): hi keeps the
-// top bfloat16 bits, lo = w - hi is itself a bfloat16 number.
-__device__ __forceinline__ void split_pair(float w0, float w1, uint32_t& hi, uint32_t& lo) {
-  const uint32_t u0 = __float_as_uint(w0), u1 = __float_as_uint(w1);
-  const uint32_t h0 = u0 & 0xFFFF0000u, h1 = u1 & 0xFFFF0000u;
-  const float l0 = __fsub_rn(w0, __uint_as_float(h0));
-  const float l1 = __fsub_rn(w1, __uint_as_float(h1));
-  hi = __byte_perm(h0, h1, 0x7632u);
-  lo = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632u);
-}
-
-// Eight weights s * (code - 8) from eight nibbles (byte i of words wa|wb, low
-// or high nibble), as hi/lo bf16 16-byte chunks.
-__device__ __forceinline__ void decode8(uint32_t wa, uint32_t wb, int sh, float s, uint4& hi,
-                                        uint4& lo) {
-  float w[8];
+// Eight decoded weights in two float2-packed halves -> one 16-byte chunk of
+// the hi tile and one of the lo tile.  A decoded weight has at most 14
+// significant bits, so hi (its top bfloat16 bits, by truncation) and
+// lo = w - hi are both exact bfloat16 numbers.
+__device__ __forceinline__ void split8(const float2 w[4], uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t word = (i < 4) ? wa : wb;
-    const uint32_t nib = (word >> (8 * (i & 3) + sh)) & 15u;
-    // (float)(nib - 8) exactly, via the 2^23 exponent bias
-    const float f = __fsub_rn(__uint_as_float(0x4B000000u | nib), 8388616.0f);
-    w[i] = __fmul_rn(s, f);
+  for (int p = 0; p < 4; ++p) {
+    const uint32_t u0 = __float_as_uint(w[p].x), u1 = __float_as_uint(w[p].y);
+    const float2 hf = make_float2(__uint_as_float(u0 & 0xFFFF0000u), __uint_as_float(u1 & 0xFFFF0000u));
+    const float2 lf = __ffma2_rn(hf, make_float2(-1.0f, -1.0f), w[p]);  // w - hi, exact
+    h[p] = __byte_perm(u0, u1, 0x7632u);
+    l[p] = __byte_perm(__float_as_uint(lf.x), __float_as_uint(lf.y), 0x7632u);
   }
-  split_pair(w[0], w[1], hi.x, lo.x);
-  split_pair(w[2], w[3], hi.y, lo.y);
-  split_pair(w[4], w[5], hi.z, lo.z);
-  split_pair(w[6], w[7], hi.w, lo.w);
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// Weights s * (code - 8) for the eight nibbles held, one per byte, in
+// (m0, m1) -- low nibbles in place (HI = false) or high nibbles left at bits
+// 4..7 (HI = true, values 16 * code).  PRMT drops each byte into the mantissa
+// of 2^23, so a float add removes the bias exactly: (2^23 + c) - (2^23 + 8)
+// = c - 8, or (2^23 + 16c) - (2^23 + 128) = 16 (c - 8) with s / 16 folded in.
+template <bool HI>
+__device__ __forceinline__ void decode8(uint32_t m0, uint32_t m1, float2 s2, uint4& hi, uint4& lo) {
+  const float bias = HI ? -8388736.0f : -8388616.0f;  // -(2^23 + 128), -(2^23 + 8)
+  const float2 b2 = make_float2(bias, bias);
+  float2 w[4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const uint32_t src = (p < 2) ? m0 : m1;
+    const uint32_t sel0 = 0x7440u | (2 * (p & 1)), sel1 = 0x7440u | (2 * (p & 1) + 1);
+    const float2 f = make_float2(__uint_as_float(__byte_perm(src, 0x4B000000u, sel0)),
+                                 __uint_as_float(__byte_perm(src, 0x4B000000u, sel1)));
+    w[p] = __fmul2_rn(__fadd2_rn(f, b2), s2);
+  }
+  split8(w, hi, lo);
 }
 
 // Store chunk c (k = 8c .. 8c+7 of the 64-wide step) of row `row` into a
@@ -140,23 +147,37 @@ __device__ __forceinline__ void st_chunk(uint32_t tile, int row, int c, uint4 v)
   *reinterpret_cast<uint4*>(gsm + off) = v;
 }
 
+// 16 code bytes at an even shared offset, as four words.
+__device__ __forceinline__ void load_codes(uint32_t qs, uint32_t q[4]) {
+  const uint32_t b = qs & ~3u;
+  const uint32_t sel = (qs & 2u) ? 0x5432u : 0x3210u;
+  uint32_t w[5];
+#pragma unroll
+  for (int i = 0; i < 5; ++i) w[i] = g_ld32(b + 4 * i);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) q[i] = __byte_perm(w[i], w[i + 1], sel);
+}
+
 // Decode one 32-weight block (scale s, 16 code bytes at `qs`) into chunks
-// c0 .. c0+3 of the hi and lo tiles.
+// c0 .. c0+3 of the hi and lo tiles: weights j and j+16 are the low and high
+// nibbles of code byte j.
 __device__ __forceinline__ void block_to_tiles(uint32_t qs, float s, uint32_t a_hi, uint32_t a_lo,
                                                int row, int c0) {
-  const uint32_t q0 = g_ld32_even(qs), q1 = g_ld32_even(qs + 4);
-  const uint32_t q2 = g_ld32_even(qs + 8), q3 = g_ld32_even(qs + 12);
+  uint32_t q[4];
+  load_codes(qs, q);
+  const float2 s1 = make_float2(s, s);
+  const float2 s16 = make_float2(s * 0.0625f, s * 0.0625f);  // exact power-of-two scaling
   uint4 h, l;
-  decode8(q0, q1, 0, s, h, l);  // weights 0..7: low nibbles of qs[0..7]
+  decode8<false>(q[0] & 0x0F0F0F0Fu, q[1] & 0x0F0F0F0Fu, s1, h, l);  // weights 0..7
   st_chunk(a_hi, row, c0 + 0, h);
   st_chunk(a_lo, row, c0 + 0, l);
-  decode8(q2, q3, 0, s, h, l);  // weights 8..15
+  decode8<false>(q[2] & 0x0F0F0F0Fu, q[3] & 0x0F0F0F0Fu, s1, h, l);  // weights 8..15
   st_chunk(a_hi, row, c0 + 1, h);
   st_chunk(a_lo, row, c0 + 1, l);
-  decode8(q0, q1, 4, s, h, l);  // weights 16..23: high nibbles of qs[0..7]
+  decode8<true>(q[0] & 0xF0F0F0F0u, q[1] & 0xF0F0F0F0u, s16, h, l);  // weights 16..23
   st_chunk(a_hi, row, c0 + 2, h);
   st_chunk(a_lo, row, c0 + 2, l);
-  decode8(q2, q3, 4, s, h, l);  // weights 24..31
+  decode8<true>(q[2] & 0xF0F0F0F0u, q[3] & 0xF0F0F0F0u, s16, h, l);  // weights 24..31
   st_chunk(a_hi, row, c0 + 3, h);
   st_chunk(a_lo, row, c0 + 3, l);
 }
@@ -175,16 +196,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
   constexpr int kBlkW = GFmt<FMT>::kBlkW, kBlkB = GFmt<FMT>::kBlkB;
   constexpr int kChunkBytes = kWChunk / kBlkW * kBlkB;  // 288 or 276
-  const Smem L = smem_layout(a.N);
+  const int kAStages = a.astages, kXStages = a.xstages;
+  const Smem L = smem_layout(a.N, kAStages, kXStages);
   const uint32_t sbase = smem_addr(gsm);
   uint64_t* bars = reinterpret_cast<uint64_t*>(gsm + L.w + kWStages * kWStageBytes);
   uint64_t* w_full = bars;
   uint64_t* w_empty = w_full + kWStages;
   uint64_t* a_full = w_empty + kWStages;
-  uint64_t* a_empty = a_full + kAStages;
-  uint64_t* x_full = a_empty + kAStages;
-  uint64_t* x_empty = x_full + kXStages;
-  uint64_t* d_full = x_empty + kXStages;
+  uint64_t* a_empty = a_full + kAStagesMax;
+  uint64_t* x_full = a_empty + kAStagesMax;
+  uint64_t* x_empty = x_full + kXStagesMax;
+  uint64_t* d_full = x_empty + kXStagesMax;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(d_full + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
@@ -197,11 +219,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&w_full[i], 1);
       mbar_init(&w_empty[i], kDequantWarps);
     }
-    for (int i = 0; i < kAStages; ++i) {
+    for (int i = 0; i < kAStagesMax; ++i) {
       mbar_init(&a_full[i], kDequantWarps);
       mbar_init(&a_empty[i], 1);
     }
-    for (int i = 0; i < kXStages; ++i) {
+    for (int i = 0; i < kXStagesMax; ++i) {
       mbar_init(&x_full[i], 1);
       mbar_init(&x_empty[i], 1);
     }
@@ -322,6 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ----------------------------------------------------------- dequant
     const int row = (warp & 3) * 32 + lane;  // TMEM lane quarter = warp % 4
+    const int half = (warp - 2) >> 2;        // which 32-weight block of each k-step
     const bool row_ok = m0 + row < a.M;
     const uintptr_t row_addr =
         reinterpret_cast<uintptr_t>(a.W) + static_cast<uintptr_t>((m0 + (row_ok ? row : 0)) * a.rowbytes);
@@ -343,32 +366,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                             static_cast<uint32_t>((row_addr + static_cast<uintptr_t>(c) * kChunkBytes) & 15u);
       const int64_t blk0 = static_cast<int64_t>(c) * (kWChunk / kBlkW);  // first block of the chunk
       if constexpr (FMT == GQ_FMT_Q4_0) {
-#pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
-          const int jb = 2 * j + bb;  // block within the chunk
-          if (blk0 + jb < nblk_row) {
-            const uint32_t o = slot + jb * 18;
-            block_to_tiles(o + 2, half_bits_to_float(g_ld16(o)), a_hi, a_lo, row, 4 * bb);
-          } else {
-            zero_chunks(a_hi, a_lo, row, 4 * bb);
-          }
+        const int jb = 2 * j + half;  // block within the chunk
+        if (blk0 + jb < nblk_row) {
+          const uint32_t o = slot + jb * 18;
+          block_to_tiles(o + 2, half_bits_to_float(g_ld16(o)), a_hi, a_lo, row, 4 * half);
+        } else {
+          zero_chunks(a_hi, a_lo, row, 4 * half);
         }
       } else {
         const int sb = j >> 2;  // super-block within the chunk
         const uint32_t o = slot + sb * 138;
         if (blk0 + sb < nblk_row) {
+          const int sub = 2 * (j & 3) + half;
           const float S = half_bits_to_float(g_ld16(o));
-#pragma unroll
-          for (int bb = 0; bb < 2; ++bb) {
-            const int sub = 2 * (j & 3) + bb;
-            const uint32_t qw = g_ld16(o + 2 + (sub & ~1));
-            const int qj = static_cast<int8_t>((qw >> (8 * (sub & 1))) & 0xFFu);
-            block_to_tiles(o + 10 + 16 * sub, __fmul_rn(S, static_cast<float>(qj)), a_hi, a_lo, row,
-                           4 * bb);
-          }
+          const uint32_t qw = g_ld16(o + 2 + (sub & ~1));
+          const int qj = static_cast<int8_t>((qw >> (8 * (sub & 1))) & 0xFFu);
+          block_to_tiles(o + 10 + 16 * sub, __fmul_rn(S, static_cast<float>(qj)), a_hi, a_lo, row,
+                         4 * half);
         } else {
-          zero_chunks(a_hi, a_lo, row, 0);
-          zero_chunks(a_hi, a_lo, row, 4);
+          zero_chunks(a_hi, a_lo, row, 4 * half);
         }
       }
       fence_proxy_async_smem();  // generic writes -> visible to the tensor core
@@ -385,7 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if (__all_sync(0xFFFFFFFFu, ok && !aborted())) {  // tcgen05.ld is warp-collective
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        for (int n0 = 0; n0 < a.N; n0 += 16) {
+        // the two warp groups share the columns: 16-column slices alternate
+        for (int n0 = 16 * half; n0 < a.N; n0 += 32) {
           uint32_t v[16];
           tmem_ld16(tmem_d + lane_base + n0, v);
           tmem_wait_ld();
@@ -409,9 +426,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-size_t gemm_smem_bytes(int N) {
-  return static_cast<size_t>(kAStages) * 2 * kATile + static_cast<size_t>(kXStages) * N * kBK * 2 +
-         static_cast<size_t>(kWStages) * kWStageBytes + 16 * sizeof(uint64_t) + 1024;
+size_t gemm_smem_bytes(int N, int astages, int xstages) {
+  return static_cast<size_t>(astages) * 2 * kATile + static_cast<size_t>(xstages) * N * kBK * 2 +
+         static_cast<size_t>(kWStages) * kWStageBytes +
+         (2 * kWStages + 2 * kAStagesMax + 2 * kXStagesMax + 4) * sizeof(uint64_t) + 1024;
+}
+
+// Deepest rings that fit: activations first (their loads wait on the MMA of
+// the slot they refill), then a third decoded-tile stage if room is left.
+void choose_stages(int N, int& astages, int& xstages) {
+  astages = 2;
+  xstages = kXStagesMax;
+  while (xstages > 2 && gemm_smem_bytes(N, astages, xstages) > static_cast<size_t>(kSmemBudget))
+    --xstages;
+  if (gemm_smem_bytes(N, 3, xstages) <= static_cast<size_t>(kSmemBudget)) astages = 3;
 }
 
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -484,13 +512,14 @@ gq_status gemm_entry(const void* W, int64_t M, int64_t K, const void* X, int xt,
   while (cols < static_cast<uint32_t>(N)) cols <<= 1;
   a.tmem_cols = cols;
 
-  const size_t smem = gemm_smem_bytes(N);
+  choose_stages(N, a.astages, a.xstages);
+  const size_t smem = gemm_smem_bytes(N, a.astages, a.xstages);
   static int configured_dev = -1;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
   if (configured_dev != dev) {
     if (cudaFuncSetAttribute(gemm_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(gemm_smem_bytes(256))) != cudaSuccess)
+                             kSmemBudget) != cudaSuccess)
       return GQ_ERR_CUDA;
     configured_dev = dev;
   }

@@ -97,6 +97,7 @@ struct GemvArgs {
   int* dev_status;
   long long budget;
   int B, ytype, nchunks, win, ngroups;  // win: chunks per activation window
+  int skip_first;  // self-test only: never fill the first stage, so waits run out
 };
 
 // ---- decode 8 codes (one 32-bit word = qs[4t..4t+3]) into four A registers
@@ -450,6 +451,13 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB) gemv_kernel(const Gemv
           ok = false;
           break;
         }
+        if (a.skip_first && issued == 0) {  // self-test: this stage never fills
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+          continue;
+        }
         const uint32_t nbytes = (c < nfull) ? static_cast<uint32_t>(kChunkBytes) : tail_bytes;
         uint32_t len = 0;
         uintptr_t lo = 0;
@@ -479,6 +487,7 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB) gemv_kernel(const Gemv
     // released, whatever the consumers did.
     if (lane == 0) {
       for (int u = max(0, issued - kStages); u < issued; ++u) {
+        if (a.skip_first && u == 0) continue;  // never issued
         if (!mbar_wait(&full[u % kStages], static_cast<uint32_t>(u / kStages) & 1u, a.budget)) {
           report(a.dev_status, GQ_DEV_TIMEOUT);
           break;
@@ -672,7 +681,8 @@ gq_status dispatch_gemv(const GemvArgs& a, cudaStream_t s, bool pdl) {
 
 template <int FMT>
 gq_status gemv_entry(const void* W, int64_t M, int64_t K, const void* x, int xt, int64_t B,
-                     void* y, int yt, unsigned flags, int* dev_status, void* stream) {
+                     void* y, int yt, unsigned flags, int* dev_status, void* stream,
+                     long long budget = kWaitBudget, int skip_first = 0) {
   constexpr int kBlkW = Fmt<FMT>::kBlkW, kBlkB = Fmt<FMT>::kBlkB;
   if (M < 0 || K < 0 || B < 0) return GQ_ERR_INVALID_ARG;
   if (!valid_act_dtype(xt) || !valid_act_dtype(yt)) return GQ_ERR_DTYPE;
@@ -700,11 +710,12 @@ gq_status gemv_entry(const void* W, int64_t M, int64_t K, const void* x, int xt,
   a.x = x;
   a.y = y;
   a.dev_status = dev_status;
-  a.budget = kWaitBudget;
+  a.budget = budget;
   a.B = static_cast<int>(B);
   a.ytype = yt;
   a.nchunks = static_cast<int>((K + kChunkW - 1) / kChunkW);
   a.ngroups = static_cast<int>((M + kRows - 1) / kRows);
+  a.skip_first = skip_first;
   const int terms = (xt == GQ_F32) ? 3 : 1;
   int win = kXSmemMax / (terms * a.B * kXStride);
   if (win < 1) win = 1;
@@ -737,6 +748,17 @@ GQ_API gq_status gq_gemv_ksb(const void* W, int64_t M, int64_t K, const void* x,
                              void* stream) {
   return gq::gemv_entry<GQ_FMT_KSB>(W, M, K, x, x_dtype, B, y, y_dtype, flags, dev_status,
                                     stream);
+}
+
+// Bounded-wait self-test: a Q4_0 GEMV (fp16 x and y, batch 1) whose producer
+// never fills its first stage; with a ~1 ms budget the consumers' wait runs
+// out, the kernel ORs GQ_DEV_TIMEOUT into *dev_status, lets every copy it did
+// issue land, and exits.  Nothing faults, traps or hangs.
+GQ_API gq_status gq_selftest_gemv_timeout(const void* W, int64_t M, int64_t K, const void* x,
+                                          void* y, int* dev_status, void* stream) {
+  if (!dev_status) return GQ_ERR_INVALID_ARG;
+  return gq::gemv_entry<GQ_FMT_Q4_0>(W, M, K, x, GQ_F16, 1, y, GQ_F16, 0u, dev_status, stream,
+                                     2000000LL, 1);
 }
 
 }  // extern "C"

@@ -153,6 +153,16 @@ GQ_API gq_status gq_gemv_ksb(const void* W, int64_t M, int64_t K,
                              void* y, int y_dtype, unsigned flags,
                              int* dev_status, void* stream);
 
+/* Self-test of the bounded waits (no counterpart on the pages): runs the
+ * Q4_0 GEMV (fp16 x and y, batch 1) on the given buffers with a producer that
+ * never fills its first pipeline stage and a ~1 ms wait budget.  The consumer
+ * waits run out; the kernel ORs GQ_DEV_TIMEOUT into *dev_status (required),
+ * lets the copies it did issue land and exits; y is unspecified.  Nothing
+ * faults, traps or hangs, and the context stays usable.  Arguments as for
+ * gq_gemv_q4_0. */
+GQ_API gq_status gq_selftest_gemv_timeout(const void* W, int64_t M, int64_t K, const void* x,
+                                          void* y, int* dev_status, void* stream);
+
 /* Dequantize-fused batched product for batches that make a dense
  * contraction: Y = W_hat * X^T on the tcgen05 tensor cores (the matrix
  * multiply that consumes decoded blocks, Q4_0 chapter 4.3).

@@ -12,6 +12,14 @@ GOLDEN = os.path.join(ROOT, "tests", "golden")
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+    # the CUDA library and the oracle must exist before the tests import them
+    if not os.path.exists(os.path.join(ROOT, "bit_gemv_q4_b200", "libgq.so")):
+        import importlib.util
+        spec = importlib.util.spec_from_file_location(
+            "gq_library_build", os.path.join(ROOT, "bit_gemv_q4_b200", "build.py"))
+        mod = importlib.util.module_from_spec(spec)
+        spec.loader.exec_module(mod)
+        mod.build()
 
 
 def pytest_collection_modifyitems(config, items):
