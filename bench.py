@@ -195,14 +195,25 @@ def build_gemv_set(gq, synth, copies, device, pdl=True):
         x = synth.activations(1, K, seed=200 + ci, dtype=torch.float16, device=device)
         y = torch.empty((1, M), dtype=torch.float16, device=device)
         gemv = gq.gq_gemv_q4_0 if fmt == "q4_0" else gq.gq_gemv_ksb
-        sets.append(dict(fmt=fmt, M=M, K=K, W=Wc, x=x, y=y, gemv=gemv, nbytes=nb))
+        sets.append(dict(fmt=fmt, M=M, K=K, W=Wc, x=x, y=y, gemv=gemv, nbytes=nb, ws=None,
+                         kernels=1))
     torch.cuda.synchronize()
     return sets
 
 
+def gemv_workspace(gq, fmt, M, K, B, xdtype, device):
+    """A zeroed workspace for gq_gemv_* (None when the case needs none).  The
+    calls of one stream run in order, so they could share one."""
+    import torch
+    code = gq.GQ_FMT_Q4_0 if fmt == "q4_0" else gq.GQ_FMT_KSB
+    need = gq.gq_gemv_workspace_bytes(code, M, K, B, xdtype)
+    return torch.zeros(need, dtype=torch.uint8, device=device) if need else None
+
+
 def launch_case(gq, s, copies, flags):
     for c in range(copies):
-        s["gemv"](s["W"][c], s["M"], s["K"], s["x"], y_dtype=s["y"].dtype, out=s["y"], flags=flags)
+        s["gemv"](s["W"][c], s["M"], s["K"], s["x"], y_dtype=s["y"].dtype, out=s["y"], flags=flags,
+                  workspace=s["ws"])
 
 
 def capture(fn):
@@ -245,7 +256,7 @@ def run_ours(args, rank, ws, local):
     flags = gq.GQ_GEMV_PDL
     wbytes_step = sum(s["nbytes"] for s in sets) * copies
     algo_bytes_step = sum(s["nbytes"] + s["K"] * 2 + s["M"] * 2 for s in sets) * copies
-    launches_step = len(sets) * copies
+    launches_step = sum(s["kernels"] for s in sets) * copies
 
     def step():
         for s in sets:
@@ -450,12 +461,16 @@ def run_suite(path):
         return (gq.gq_quantize_q4_0 if fmt == "q4_0" else gq.gq_quantize_ksb)(w.view(-1))
 
     # --- single GEMVs (decode shapes), cold weights, graph + PDL
-    for fmt, M, K, B, xdt, ydt, name in (
-            ("q4_0", 256, 1024, 1, torch.float32, torch.float32, "tiny 256x1024 fp32"),
-            ("q4_0", 4096, 4096, 1, torch.float16, torch.float16, "decode 4096x4096"),
-            ("ksb", 11008, 4096, 1, torch.float16, torch.float16, "MLP 11008x4096 ksb B=1"),
-            ("ksb", 11008, 4096, 8, torch.float16, torch.float16, "MLP 11008x4096 ksb B=8"),
-            ("q4_0", 11008, 4096, 8, torch.float16, torch.float16, "MLP 11008x4096 q4_0 B=8")):
+    for fmt, M, K, B, xdt, ydt, name, use_ws in (
+            ("q4_0", 256, 1024, 1, torch.float32, torch.float32, "tiny 256x1024 fp32", False),
+            ("q4_0", 4096, 4096, 1, torch.float16, torch.float16, "decode 4096x4096", False),
+            ("ksb", 11008, 4096, 1, torch.float16, torch.float16, "MLP 11008x4096 ksb B=1", False),
+            ("ksb", 11008, 4096, 8, torch.float16, torch.float16, "MLP 11008x4096 ksb B=8", False),
+            ("q4_0", 11008, 4096, 8, torch.float16, torch.float16, "MLP 11008x4096 q4_0 B=8", False),
+            # the batch-1 integer tensor-core path (workspace given), for comparison
+            ("q4_0", 4096, 4096, 1, torch.float16, torch.float16, "decode 4096x4096, integer path", True),
+            ("q4_0", 4096, 11008, 1, torch.float16, torch.float16, "4096x11008, integer path", True),
+            ("q4_0", 11008, 4096, 1, torch.float16, torch.float16, "11008x4096, integer path", True)):
         w = synth.gaussian_weights(M, K, seed=7, device=dev)
         q = quant(fmt, w)
         del w
@@ -466,8 +481,10 @@ def run_suite(path):
         x = synth.activations(B, K, seed=8, dtype=xdt, device=dev)
         y = torch.empty((B, M), dtype=ydt, device=dev)
         f = gq.gq_gemv_q4_0 if fmt == "q4_0" else gq.gq_gemv_ksb
+        wsp = gemv_workspace(gq, fmt, M, K, B, xdt, dev) if use_ws else None
         ms = _graph_ms_per_launch(
-            lambda: [f(Wc[i], M, K, x, y_dtype=ydt, out=y, flags=gq.GQ_GEMV_PDL) for i in range(copies)],
+            lambda: [f(Wc[i], M, K, x, y_dtype=ydt, out=y, flags=gq.GQ_GEMV_PDL, workspace=wsp)
+                     for i in range(copies)],
             copies, 20)
         emit({"row": "gemv", "workload": name, "format": fmt, "M": M, "K": K, "B": B,
               "us": round(ms * 1e3, 3), "weight_gbs": round(nb / (ms * 1e-3) / 1e9, 1),
@@ -489,8 +506,10 @@ def run_suite(path):
         x = synth.activations(1, 4096, seed=9, dtype=torch.float16, device=dev)
         ys = {M: torch.empty((1, M), dtype=torch.float16, device=dev) for M in (4096, 11008)}
         f = gq.gq_gemv_q4_0 if fmt == "q4_0" else gq.gq_gemv_ksb
+        wss = {M: None for M in (4096, 11008)}
         ms = _graph_ms_per_launch(
-            lambda: [f(qm, M, K, x, out=ys[M], flags=gq.GQ_GEMV_PDL) for qm, M, K in mats], 1, 5)
+            lambda: [f(qm, M, K, x, out=ys[M], flags=gq.GQ_GEMV_PDL, workspace=wss[M])
+                     for qm, M, K in mats], 1, 5)
         emit({"row": "model_stream", "workload": "32 layers x (4 x 4096x4096 + 3 x 11008x4096), "
               "224 batch-1 GEMVs, one CUDA graph", "format": fmt, "weight_bytes": total,
               "ms": round(ms, 3), "weight_gbs": round(total / (ms * 1e-3) / 1e9, 1),
@@ -544,7 +563,7 @@ def run_suite(path):
     out.close()
 
 
-def run_single(spec, launches, batch, flags):
+def run_single(spec, launches, batch, flags, use_ws=False):
     """A few launches of one product on distinct copies of one matrix (for
     profilers): spec = "gemv:q4_0:4096:11008" or "gemm:ksb:11008:4096"."""
     import torch
@@ -564,7 +583,8 @@ def run_single(spec, launches, batch, flags):
         x = synth.activations(batch, K, seed=2, dtype=torch.float16, device=dev)
         f = gq.gq_gemv_q4_0 if fmt == "q4_0" else gq.gq_gemv_ksb
         y = torch.empty((batch, M), dtype=torch.float16, device=dev)
-        run = lambda i: f(Wc[i % copies], M, K, x, out=y, flags=flags)
+        wsp = gemv_workspace(gq, fmt, M, K, batch, torch.float16, dev) if use_ws else None
+        run = lambda i: f(Wc[i % copies], M, K, x, out=y, flags=flags, workspace=wsp)
     else:
         x = synth.activations(batch, K, seed=2, dtype=torch.bfloat16, device=dev)
         f = gq.gq_gemm_q4_0 if fmt == "q4_0" else gq.gq_gemm_ksb
@@ -592,9 +612,11 @@ def main():
     ap.add_argument("--launches", type=int, default=4)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--flags", type=int, default=0)
+    ap.add_argument("--workspace", action="store_true",
+                    help="--single gemv: pass a workspace (the batch-1 integer path)")
     args = ap.parse_args()
     if args.single:
-        run_single(args.single, args.launches, args.batch, args.flags)
+        run_single(args.single, args.launches, args.batch, args.flags, args.workspace)
         return
 
     rank, ws, local = dist_setup()

@@ -30,7 +30,7 @@ EXPORTS = (
     "gq_q4_0_bytes", "gq_ksb_bytes",
     "gq_quantize_q4_0", "gq_quantize_ksb",
     "gq_dequantize_q4_0", "gq_dequantize_ksb",
-    "gq_gemv_q4_0", "gq_gemv_ksb",
+    "gq_gemv_workspace_bytes", "gq_gemv_q4_0", "gq_gemv_ksb",
     "gq_gemm_workspace_bytes", "gq_gemm_q4_0", "gq_gemm_ksb",
     "gq_selftest_gemv_timeout",
 )
@@ -67,9 +67,12 @@ def _load() -> ctypes.CDLL:
         f = getattr(L, name)
         f.argtypes = [vp, i64, vp, vp]
         f.restype = c_int
+    L.gq_gemv_workspace_bytes.argtypes = [c_int, i64, i64, i64, c_int]
+    L.gq_gemv_workspace_bytes.restype = ctypes.c_size_t
     for name in ("gq_gemv_q4_0", "gq_gemv_ksb"):
         f = getattr(L, name)
-        f.argtypes = [vp, i64, i64, vp, c_int, i64, vp, c_int, c_uint, vp, vp]
+        f.argtypes = [vp, i64, i64, vp, c_int, i64, vp, c_int, vp, ctypes.c_size_t, c_uint, vp,
+                      vp]
         f.restype = c_int
     L.gq_gemm_workspace_bytes.argtypes = [c_int, i64, i64, i64]
     L.gq_gemm_workspace_bytes.restype = ctypes.c_size_t
@@ -165,8 +168,27 @@ def gq_dequantize_ksb(q: torch.Tensor, n: int, out: torch.Tensor | None = None,
     return _dequantize("gq_dequantize_ksb", q, n, out, stream)
 
 
-def _gemv(name: str, W: torch.Tensor, M: int, K: int, x: torch.Tensor, y_dtype, out,
-          flags: int, dev_status, stream):
+def gq_gemv_workspace_bytes(fmt: int, M: int, K: int, B: int, x_dtype) -> int:
+    code = _DTYPE_CODE[x_dtype] if isinstance(x_dtype, torch.dtype) else int(x_dtype)
+    return int(lib.gq_gemv_workspace_bytes(int(fmt), int(M), int(K), int(B), code))
+
+
+# Zeroed GEMV workspaces, one per (device, stream): calls on one stream run in
+# order, and each successful call leaves the workspace ready for the next.
+_gemv_ws: dict = {}
+
+
+def _gemv_workspace(need: int, device: torch.device, stream) -> torch.Tensor:
+    key = (device.index, _stream(stream))
+    ws = _gemv_ws.get(key)
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(need, dtype=torch.uint8, device=device)
+        _gemv_ws[key] = ws
+    return ws
+
+
+def _gemv(name: str, fmt: int, W: torch.Tensor, M: int, K: int, x: torch.Tensor, y_dtype, out,
+          workspace, flags: int, dev_status, stream):
     x2 = x if x.dim() == 2 else x.reshape(1, -1)
     B = x2.shape[0]
     if x2.shape[1] != K:
@@ -175,24 +197,39 @@ def _gemv(name: str, W: torch.Tensor, M: int, K: int, x: torch.Tensor, y_dtype, 
         raise TypeError("activations and outputs must be float32, float16 or bfloat16")
     if out is None:
         out = torch.empty((B, M), dtype=y_dtype, device=x2.device)
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError("workspace must be 'auto', None or a uint8 CUDA tensor")
+        need = gq_gemv_workspace_bytes(fmt, M, K, B, x2.dtype)
+        workspace = _gemv_workspace(need, x2.device, stream) if need else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(getattr(lib, name)(_ptr(W), int(M), int(K), _ptr(x2), _DTYPE_CODE[x2.dtype], B,
-                              _ptr(out), _DTYPE_CODE[out.dtype], int(flags), _ptr(dev_status),
-                              _stream(stream)), name)
+                              _ptr(out), _DTYPE_CODE[out.dtype], _ptr(workspace), ws_bytes,
+                              int(flags), _ptr(dev_status), _stream(stream)), name)
     return out
 
 
 def gq_gemv_q4_0(W: torch.Tensor, M: int, K: int, x: torch.Tensor, y_dtype=torch.float16,
                  out: torch.Tensor | None = None, flags: int = 0,
-                 dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """y[B, M] = W_hat[M, K] @ x[B, K]^T for Q4_0 weights; B in 1..8."""
-    return _gemv("gq_gemv_q4_0", W, M, K, x, y_dtype, out, flags, dev_status, stream)
+                 dev_status: torch.Tensor | None = None, stream=None,
+                 workspace=None) -> torch.Tensor:
+    """y[B, M] = W_hat[M, K] @ x[B, K]^T for Q4_0 weights; B in 1..8.
+
+    workspace: None (the default path), "auto" (a zeroed scratch buffer cached
+    per device and stream) or a uint8 CUDA tensor of at least
+    gq_gemv_workspace_bytes(...) bytes, zero before its first use; with a
+    workspace, batch-1 fp16 calls take the integer tensor-core path."""
+    return _gemv("gq_gemv_q4_0", GQ_FMT_Q4_0, W, M, K, x, y_dtype, out, workspace, flags,
+                 dev_status, stream)
 
 
 def gq_gemv_ksb(W: torch.Tensor, M: int, K: int, x: torch.Tensor, y_dtype=torch.float16,
                 out: torch.Tensor | None = None, flags: int = 0,
-                dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+                dev_status: torch.Tensor | None = None, stream=None,
+                workspace=None) -> torch.Tensor:
     """y[B, M] = W_hat[M, K] @ x[B, K]^T for super-block weights; B in 1..8."""
-    return _gemv("gq_gemv_ksb", W, M, K, x, y_dtype, out, flags, dev_status, stream)
+    return _gemv("gq_gemv_ksb", GQ_FMT_KSB, W, M, K, x, y_dtype, out, workspace, flags,
+                 dev_status, stream)
 
 
 def gq_gemm_workspace_bytes(fmt: int, M: int, K: int, B: int) -> int:

@@ -442,23 +442,6 @@ void choose_stages(int N, int& astages, int& xstages) {
   if (gemm_smem_bytes(N, 3, xstages) <= static_cast<size_t>(kSmemBudget)) astages = 3;
 }
 
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled encode_fn() {
-  static EncodeTiled fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiled>(p);
-  }
-  return fn;
-}
-
 template <int FMT>
 gq_status gemm_entry(const void* W, int64_t M, int64_t K, const void* X, int xt, int64_t B, void* Y,
                      int yt, void* workspace, size_t ws_bytes, int* dev_status, void* stream) {
@@ -482,7 +465,7 @@ gq_status gemm_entry(const void* W, int64_t M, int64_t K, const void* X, int xt,
   if (misaligned16(W) || misaligned16(X)) return GQ_ERR_ALIGNMENT;
   if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return GQ_ERR_ALIGNMENT;
 
-  EncodeTiled enc = encode_fn();
+  EncodeTiled enc = tensor_map_encoder();
   if (!enc) return GQ_ERR_CUDA;
   const int N = static_cast<int>((B + 15) / 16 * 16);
   CUtensorMap xmap;

@@ -41,6 +41,7 @@
 
 #include "gq.h"
 #include "gq_device.cuh"
+#include "gq_gemv_i8.h"
 #include "gq_host.h"
 
 namespace gq {
@@ -681,8 +682,9 @@ gq_status dispatch_gemv(const GemvArgs& a, cudaStream_t s, bool pdl) {
 
 template <int FMT>
 gq_status gemv_entry(const void* W, int64_t M, int64_t K, const void* x, int xt, int64_t B,
-                     void* y, int yt, unsigned flags, int* dev_status, void* stream,
-                     long long budget = kWaitBudget, int skip_first = 0) {
+                     void* y, int yt, void* workspace, size_t ws_bytes, unsigned flags,
+                     int* dev_status, void* stream, long long budget = kWaitBudget,
+                     int skip_first = 0) {
   constexpr int kBlkW = Fmt<FMT>::kBlkW, kBlkB = Fmt<FMT>::kBlkB;
   if (M < 0 || K < 0 || B < 0) return GQ_ERR_INVALID_ARG;
   if (!valid_act_dtype(xt) || !valid_act_dtype(yt)) return GQ_ERR_DTYPE;
@@ -724,6 +726,8 @@ gq_status gemv_entry(const void* W, int64_t M, int64_t K, const void* x, int xt,
 
   const bool pdl = (flags & GQ_GEMV_PDL) != 0;
   cudaStream_t s = as_stream(stream);
+  if (workspace && ws_bytes && !skip_first && i8_eligible(FMT, M, K, B, xt, W))
+    return i8_gemv(W, M, K, x, y, yt, workspace, ws_bytes, pdl, dev_status, s);
   switch (xt) {
     case GQ_F16: return dispatch_gemv<FMT, XT_F16>(a, s, pdl);
     case GQ_BF16: return dispatch_gemv<FMT, XT_BF16>(a, s, pdl);
@@ -736,18 +740,26 @@ gq_status gemv_entry(const void* W, int64_t M, int64_t K, const void* x, int xt,
 
 extern "C" {
 
+GQ_API size_t gq_gemv_workspace_bytes(int fmt, int64_t M, int64_t K, int64_t B, int x_dtype) {
+  if (M <= 0 || K <= 0) return 0;
+  // eligibility apart from the pointer: a 16-byte-aligned stand-in
+  if (!gq::i8_eligible(fmt, M, K, B, x_dtype, reinterpret_cast<const void*>(uintptr_t{16})))
+    return 0;
+  return gq::i8_workspace_bytes(M, K);
+}
+
 GQ_API gq_status gq_gemv_q4_0(const void* W, int64_t M, int64_t K, const void* x, int x_dtype,
-                              int64_t B, void* y, int y_dtype, unsigned flags, int* dev_status,
-                              void* stream) {
-  return gq::gemv_entry<GQ_FMT_Q4_0>(W, M, K, x, x_dtype, B, y, y_dtype, flags, dev_status,
-                                     stream);
+                              int64_t B, void* y, int y_dtype, void* workspace, size_t ws_bytes,
+                              unsigned flags, int* dev_status, void* stream) {
+  return gq::gemv_entry<GQ_FMT_Q4_0>(W, M, K, x, x_dtype, B, y, y_dtype, workspace, ws_bytes,
+                                     flags, dev_status, stream);
 }
 
 GQ_API gq_status gq_gemv_ksb(const void* W, int64_t M, int64_t K, const void* x, int x_dtype,
-                             int64_t B, void* y, int y_dtype, unsigned flags, int* dev_status,
-                             void* stream) {
-  return gq::gemv_entry<GQ_FMT_KSB>(W, M, K, x, x_dtype, B, y, y_dtype, flags, dev_status,
-                                    stream);
+                             int64_t B, void* y, int y_dtype, void* workspace, size_t ws_bytes,
+                             unsigned flags, int* dev_status, void* stream) {
+  return gq::gemv_entry<GQ_FMT_KSB>(W, M, K, x, x_dtype, B, y, y_dtype, workspace, ws_bytes,
+                                    flags, dev_status, stream);
 }
 
 // Bounded-wait self-test: a Q4_0 GEMV (fp16 x and y, batch 1) whose producer
@@ -757,8 +769,8 @@ GQ_API gq_status gq_gemv_ksb(const void* W, int64_t M, int64_t K, const void* x,
 GQ_API gq_status gq_selftest_gemv_timeout(const void* W, int64_t M, int64_t K, const void* x,
                                           void* y, int* dev_status, void* stream) {
   if (!dev_status) return GQ_ERR_INVALID_ARG;
-  return gq::gemv_entry<GQ_FMT_Q4_0>(W, M, K, x, GQ_F16, 1, y, GQ_F16, 0u, dev_status, stream,
-                                     2000000LL, 1);
+  return gq::gemv_entry<GQ_FMT_Q4_0>(W, M, K, x, GQ_F16, 1, y, GQ_F16, nullptr, 0, 0u,
+                                     dev_status, stream, 2000000LL, 1);
 }
 
 }  // extern "C"

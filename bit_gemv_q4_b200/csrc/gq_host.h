@@ -3,6 +3,7 @@
 // the launch wrapper.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -20,6 +21,13 @@ inline int dtype_size(int t) { return t == GQ_F32 ? 4 : 2; }
 
 // Number of SMs of the current device (looked up once per device).
 int sm_count();
+
+// cuTensorMapEncodeTiled from the driver (looked up once; null if missing).
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiled tensor_map_encoder();
 
 // cudaLaunchKernelEx wrapper; `pdl` adds programmatic stream serialization.
 template <typename... KArgs, typename... Args>

@@ -142,16 +142,33 @@ GQ_API gq_status gq_dequantize_ksb(const void* q, int64_t n, float* out, void* s
  *   B: 1..8 (0 launches nothing).
  * Arithmetic: products of the exact decoded weights with the exact inputs
  * (fp32 x is split exactly into three bfloat16 terms), accumulated in fp32,
- * rounded once to y_dtype.  flags: 0 or GQ_GEMV_PDL.  dev_status: optional,
- * receives GQ_DEV_TIMEOUT if a pipeline wait ever gives up. */
+ * rounded once to y_dtype.
+ * workspace / ws_bytes: optional caller-owned device scratch of at least
+ *   gq_gemv_workspace_bytes(...) bytes (a size that does not depend on M or
+ *   K), 256-byte aligned, all zero before its first use.  When that size is
+ *   nonzero and a workspace is given, the call takes the batch-1 integer
+ *   tensor-core path: x is split exactly into six signed 7-bit digit columns
+ *   (every fp16 value is an integer multiple of 2^-24 below 2^16), the codes
+ *   are multiplied as unsigned bytes with exact int32 sums, and only the fp32
+ *   accumulation rounds.  The work is split evenly over the SMs; rows shared
+ *   by two SMs are combined in a fixed order, so results do not depend on
+ *   scheduling.  A successful call leaves the workspace ready for the next
+ *   call (of any shape); after a call that fails or reports GQ_DEV_TIMEOUT,
+ *   zero it again.  Calls that may run at the same time need separate
+ *   workspaces.  NULL (or a size of 0) selects the path above.  A NaN or
+ *   infinite x element makes every output of that path NaN (and sets
+ *   GQ_DEV_NONFINITE).
+ * flags: 0 or GQ_GEMV_PDL.  dev_status: optional, receives GQ_DEV_TIMEOUT if
+ * a pipeline wait ever gives up. */
+GQ_API size_t gq_gemv_workspace_bytes(int fmt, int64_t M, int64_t K, int64_t B, int x_dtype);
 GQ_API gq_status gq_gemv_q4_0(const void* W, int64_t M, int64_t K,
                               const void* x, int x_dtype, int64_t B,
-                              void* y, int y_dtype, unsigned flags,
-                              int* dev_status, void* stream);
+                              void* y, int y_dtype, void* workspace, size_t ws_bytes,
+                              unsigned flags, int* dev_status, void* stream);
 GQ_API gq_status gq_gemv_ksb(const void* W, int64_t M, int64_t K,
                              const void* x, int x_dtype, int64_t B,
-                             void* y, int y_dtype, unsigned flags,
-                             int* dev_status, void* stream);
+                             void* y, int y_dtype, void* workspace, size_t ws_bytes,
+                             unsigned flags, int* dev_status, void* stream);
 
 /* Self-test of the bounded waits (no counterpart on the pages): runs the
  * Q4_0 GEMV (fp16 x and y, batch 1) on the given buffers with a producer that

@@ -82,12 +82,13 @@ def test_dequantize_validation(name, block):
 def test_gemv_validation(name, block):
     f = getattr(gq.lib, name)
     K = 4 * block
-    ok = dict(W=A, M=64, K=K, x=A, xt=1, B=1, y=A, yt=1, flags=0, st=None, s=None)
+    ok = dict(W=A, M=64, K=K, x=A, xt=1, B=1, y=A, yt=1, ws=None, wsb=0, flags=0, st=None,
+              s=None)
 
     def call(**kw):
         a = dict(ok, **kw)
-        return f(a["W"], a["M"], a["K"], a["x"], a["xt"], a["B"], a["y"], a["yt"], a["flags"],
-                 a["st"], a["s"])
+        return f(a["W"], a["M"], a["K"], a["x"], a["xt"], a["B"], a["y"], a["yt"], a["ws"],
+                 a["wsb"], a["flags"], a["st"], a["s"])
 
     assert call(M=-1) == INVALID
     assert call(K=-block) == INVALID
@@ -139,3 +140,22 @@ def test_gemm_validation(name, block):
     assert call(X=A + 8) == ALIGN
     assert call(st=A + 1) == ALIGN
     assert gq.gq_gemm_workspace_bytes(0, 11008, 4096, 256) >= 0
+
+
+def test_gemv_workspace_sizes_and_checks():
+    f = gq.lib.gq_gemv_q4_0
+    Q40, KSB = gq.GQ_FMT_Q4_0, gq.GQ_FMT_KSB
+    need = gq.gq_gemv_workspace_bytes(Q40, 4096, 11008, 1, gq.GQ_F16)
+    # counts and partial sums of the SMs; the same for every eligible shape
+    assert need > 0
+    assert gq.gq_gemv_workspace_bytes(Q40, 17, 256, 1, gq.GQ_F16) == need
+    # only batch-1 fp16 Q4_0 with K % 256 == 0 uses a workspace
+    assert gq.gq_gemv_workspace_bytes(Q40, 4096, 11008, 2, gq.GQ_F16) == 0
+    assert gq.gq_gemv_workspace_bytes(Q40, 4096, 11008, 1, gq.GQ_BF16) == 0
+    assert gq.gq_gemv_workspace_bytes(Q40, 4096, 288, 1, gq.GQ_F16) == 0
+    assert gq.gq_gemv_workspace_bytes(KSB, 4096, 11008, 1, gq.GQ_F16) == 0
+    assert gq.gq_gemv_workspace_bytes(Q40, 0, 4096, 1, gq.GQ_F16) == 0
+    args = (A, 4096, 11008, A, 1, 1, A, 1)
+    # too small, then misaligned: both refused before any launch
+    assert f(*args, A, need - 1, 0, None, None) == 9
+    assert f(*args, A + 16, need, 0, None, None) == ALIGN
