@@ -32,7 +32,7 @@ EXPORTS = (
     "gq_dequantize_q4_0", "gq_dequantize_ksb",
     "gq_gemv_workspace_bytes", "gq_gemv_q4_0", "gq_gemv_ksb",
     "gq_gemm_workspace_bytes", "gq_gemm_q4_0", "gq_gemm_ksb",
-    "gq_selftest_gemv_timeout",
+    "gq_selftest_gemv_timeout", "gq_gemv_q4_0_noalloc",
 )
 
 _DTYPE_CODE = {torch.float32: GQ_F32, torch.float16: GQ_F16, torch.bfloat16: GQ_BF16}
@@ -80,6 +80,8 @@ def _load() -> ctypes.CDLL:
         f = getattr(L, name)
         f.argtypes = [vp, i64, i64, vp, c_int, i64, vp, c_int, vp, ctypes.c_size_t, vp, vp]
         f.restype = c_int
+    L.gq_gemv_q4_0_noalloc.argtypes = [vp, i64, i64, vp, vp, c_int, c_uint, vp, vp]
+    L.gq_gemv_q4_0_noalloc.restype = c_int
     L.gq_selftest_gemv_timeout.argtypes = [vp, i64, i64, vp, vp, vp, vp]
     L.gq_selftest_gemv_timeout.restype = c_int
     return L
@@ -270,6 +272,21 @@ def gq_gemm_ksb(W: torch.Tensor, M: int, K: int, X: torch.Tensor, y_dtype=torch.
     """Y[B, M] = W_hat[M, K] @ X[B, K]^T for super-block weights on the tensor cores."""
     return _gemm("gq_gemm_ksb", GQ_FMT_KSB, W, M, K, X, y_dtype, out, workspace, dev_status,
                  stream)
+
+
+def gq_gemv_q4_0_noalloc(W: torch.Tensor, M: int, K: int, x: torch.Tensor, y_dtype=torch.float16,
+                         out: torch.Tensor | None = None, flags: int = 0,
+                         dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Batch-1 Q4_0 GEMV (fp16 x) on the library's static scratch."""
+    x2 = x if x.dim() == 2 else x.reshape(1, -1)
+    if x2.shape != (1, K) or x2.dtype != torch.float16:
+        raise ValueError("x must be one fp16 vector of length K")
+    if out is None:
+        out = torch.empty((1, M), dtype=y_dtype, device=x2.device)
+    _check(lib.gq_gemv_q4_0_noalloc(_ptr(W), int(M), int(K), _ptr(x2), _ptr(out),
+                                    _DTYPE_CODE[out.dtype], int(flags), _ptr(dev_status),
+                                    _stream(stream)), "gq_gemv_q4_0_noalloc")
+    return out
 
 
 def gq_selftest_gemv_timeout(W: torch.Tensor, M: int, K: int, x: torch.Tensor, y: torch.Tensor,

@@ -762,6 +762,25 @@ GQ_API gq_status gq_gemv_ksb(const void* W, int64_t M, int64_t K, const void* x,
                                     flags, dev_status, stream);
 }
 
+// Allocation-free batch-1 Q4_0 GEMV: the integer tensor-core path of
+// gq_gemv_q4_0 with its scratch in a static device array, for callers that
+// cannot hand the library device memory -- a runtime that allocates nothing
+// after start-up, or a C caller with no device allocator of its own.
+GQ_API gq_status gq_gemv_q4_0_noalloc(const void* W, int64_t M, int64_t K, const void* x,
+                                      void* y, int y_dtype, unsigned flags, int* dev_status,
+                                      void* stream) {
+  if (M < 0 || K < 0) return GQ_ERR_INVALID_ARG;
+  if (!gq::valid_act_dtype(y_dtype)) return GQ_ERR_DTYPE;
+  if (flags & ~GQ_GEMV_PDL) return GQ_ERR_INVALID_ARG;
+  if (M == 0) return GQ_OK;
+  if (!W || !x || !y) return GQ_ERR_INVALID_ARG;
+  if (gq::misaligned16(W) || gq::misaligned16(x) || gq::misaligned16(y)) return GQ_ERR_ALIGNMENT;
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return GQ_ERR_ALIGNMENT;
+  if (!gq::i8_eligible(GQ_FMT_Q4_0, M, K, 1, GQ_F16, W)) return GQ_ERR_SHAPE;
+  return gq::i8_gemv_noalloc(W, M, K, x, y, y_dtype, (flags & GQ_GEMV_PDL) != 0, dev_status,
+                             gq::as_stream(stream));
+}
+
 // Bounded-wait self-test: a Q4_0 GEMV (fp16 x and y, batch 1) whose producer
 // never fills its first stage; with a ~1 ms budget the consumers' wait runs
 // out, the kernel ORs GQ_DEV_TIMEOUT into *dev_status, lets every copy it did

@@ -570,6 +570,10 @@ Split make_split(int64_t M, int64_t K) {
   return sp;
 }
 
+// Scratch of gq_gemv_q4_0_noalloc: the same counts and partial sums as a
+// caller's workspace, in static device memory instead.
+__device__ __align__(256) uint8_t g_noalloc_scratch[kWsBytes];
+
 }  // namespace
 
 bool i8_eligible(int fmt, int64_t M, int64_t K, int64_t B, int xt, const void* W) {
@@ -630,6 +634,36 @@ gq_status i8_gemv(const void* W, int64_t M, int64_t K, const void* x, void* y, i
   a.budget = kWaitBudget;
   const size_t smem = fixed_smem(nblk) + static_cast<size_t>(nst) * kStageBytes;
   return launch(gemv_i8_kernel, dim3(sp.P), dim3(kThreads), smem, stream, pdl, wmap, a);
+}
+
+}  // namespace gq
+
+namespace gq {
+
+// Address of the static scratch on the current device, looked up once per
+// device (the first call on a device should come before any stream capture).
+static gq_status noalloc_scratch(uint8_t** out) {
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GQ_ERR_CUDA;
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GQ_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = static_cast<uint8_t*>(addr[dev]);
+  return GQ_OK;
+}
+
+gq_status i8_gemv_noalloc(const void* W, int64_t M, int64_t K, const void* x, void* y, int yt,
+                          bool pdl, int* dev_status, cudaStream_t stream) {
+  if (make_split(M, K).P > kMaxCtas) return GQ_ERR_WORKSPACE;  // beyond the static scratch
+  uint8_t* scratch = nullptr;
+  const gq_status st = noalloc_scratch(&scratch);
+  if (st != GQ_OK) return st;
+  // the counts must start at zero: clear them in stream order before the launch
+  if (cudaMemsetAsync(scratch, 0, kCountersBytes, stream) != cudaSuccess) return GQ_ERR_CUDA;
+  return i8_gemv(W, M, K, x, y, yt, scratch, kWsBytes, pdl, dev_status, stream);
 }
 
 }  // namespace gq

@@ -18,9 +18,14 @@ bool i8_eligible(int fmt, int64_t M, int64_t K, int64_t B, int xt, const void* W
 // Workspace bytes of that path for an M x K matrix on the current device.
 size_t i8_workspace_bytes(int64_t M, int64_t K);
 
-// Launches the activation split and the GEMV on `stream`.
+// Launches the GEMV (it splits x itself) on `stream`.
 gq_status i8_gemv(const void* W, int64_t M, int64_t K, const void* x, void* y, int yt,
                   void* workspace, size_t ws_bytes, bool pdl, int* dev_status,
                   cudaStream_t stream);
+
+// The same path with static device scratch instead of a workspace (the
+// counts are cleared in stream order before each launch).
+gq_status i8_gemv_noalloc(const void* W, int64_t M, int64_t K, const void* x, void* y, int yt,
+                          bool pdl, int* dev_status, cudaStream_t stream);
 
 }  // namespace gq

@@ -170,6 +170,24 @@ GQ_API gq_status gq_gemv_ksb(const void* W, int64_t M, int64_t K,
                              void* y, int y_dtype, void* workspace, size_t ws_bytes,
                              unsigned flags, int* dev_status, void* stream);
 
+/* Allocation-free variant (no counterpart on the pages): the batch-1 integer
+ * tensor-core path of gq_gemv_q4_0 (fp16 x, B = 1) with its scratch -- the
+ * per-CTA counts and partial sums, 33 KB -- in a static device array of the
+ * library instead of a caller workspace.  For callers that cannot give the
+ * library device memory.  The counts are cleared with an asynchronous memset
+ * on `stream` before each launch; the library allocates nothing.
+ *   Arguments as for gq_gemv_q4_0 with x_dtype = GQ_F16, B = 1 and no
+ *   workspace.  K must be a multiple of 256 and at most 14336
+ *   (GQ_ERR_SHAPE otherwise); more SMs than the scratch covers (256) gives
+ *   GQ_ERR_WORKSPACE.
+ *   The scratch is one per device: calls that may overlap (other streams,
+ *   other host threads) race on it and must be serialised by the caller.
+ *   The first call on a device looks the scratch up with
+ *   cudaGetSymbolAddress; make it before capturing work into a graph. */
+GQ_API gq_status gq_gemv_q4_0_noalloc(const void* W, int64_t M, int64_t K, const void* x,
+                                      void* y, int y_dtype, unsigned flags, int* dev_status,
+                                      void* stream);
+
 /* Self-test of the bounded waits (no counterpart on the pages): runs the
  * Q4_0 GEMV (fp16 x and y, batch 1) on the given buffers with a producer that
  * never fills its first pipeline stage and a ~1 ms wait budget.  The consumer
