@@ -13,8 +13,10 @@
 //
 // Design (sm_100a, one 128-row tile of W per CTA, all of the batch as N):
 //  * warp 0 (producer): streams the tile's packed rows, 512 weights per row
-//    per stage, with one 1-D bulk copy per row (no multicast), and the X
-//    k-slices (64 x N bf16) with a 2-D TMA load in the 128-byte swizzle;
+//    per stage -- one 2-D TMA load of 128 rows x 304 bytes when rows are
+//    whole 16-byte granules, else one 1-D bulk copy per row (no multicast)
+//    -- and the X k-slices (64 x N bf16) with a 2-D TMA load in the
+//    128-byte swizzle;
 //  * warps 2..5 (dequant, one thread per W row): decode each 64-weight
 //    k-step into the hi and lo bf16 tiles, written straight into the
 //    K-major 128-byte-swizzled UMMA layout, then fence the async proxy;
@@ -42,8 +44,8 @@ namespace {
 constexpr int kBM = 128;                       // W rows per tile (UMMA M)
 constexpr int kBK = 64;                        // k per A/X stage (128-byte bf16 rows)
 constexpr int kWChunk = 512;                   // weights per W row per stage
-constexpr int kWPitch = 304;                   // >= 288 + 14, multiple of 16
-constexpr int kWStageBytes = kBM * kWPitch + 16;
+constexpr int kWPitch = 304;                   // 19 granules >= 12 + 288
+constexpr int kWStageBytes = kBM * kWPitch;    // 38 KB, a multiple of 1024
 constexpr int kWStages = 2;
 constexpr int kAStagesMax = 3;                 // decoded hi/lo tile pairs
 constexpr int kXStagesMax = 8;                 // activation k-slices
@@ -73,6 +75,7 @@ struct GemmArgs {
   int B, N, ytype, nsteps, nchunks;
   int astages, xstages;  // ring depths chosen from the shared-memory budget
   uint32_t tmem_cols;
+  int w_tma;             // rows are whole 16-byte granules: one TMA load per W stage
 };
 
 struct Smem {
@@ -193,7 +196,8 @@ __device__ __forceinline__ void zero_chunks(uint32_t a_hi, uint32_t a_lo, int ro
 
 template <int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
+    gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap,
+                const GemmArgs a) {
   constexpr int kBlkW = GFmt<FMT>::kBlkW, kBlkB = GFmt<FMT>::kBlkB;
   constexpr int kChunkBytes = kWChunk / kBlkW * kBlkB;  // 288 or 276
   const int kAStages = a.astages, kXStages = a.xstages;
@@ -258,31 +262,43 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const int64_t b0 = static_cast<int64_t>(c) * (kWChunk / kBlkW);
-        const uint32_t nbytes = static_cast<uint32_t>(i64min(kWChunk / kBlkW, nblk_row - b0) * kBlkB);
-        uint32_t total = 0;
-        uintptr_t lo[4];
-        uint32_t len[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = lane + 32 * i;
-          len[i] = 0;
-          if (m0 + r < a.M) {
-            const uintptr_t src = reinterpret_cast<uintptr_t>(a.W) +
-                                  static_cast<uintptr_t>((m0 + r) * a.rowbytes + b0 * kBlkB);
-            lo[i] = src & ~static_cast<uintptr_t>(15);
-            len[i] = static_cast<uint32_t>(((src + nbytes + 15) & ~static_cast<uintptr_t>(15)) - lo[i]);
+        if (a.w_tma) {
+          // the 128 rows x 304 bytes (19 granules) that hold the chunk; rows
+          // past M and bytes past the row end read as zeros
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&w_full[s], kWStageBytes);
+            tma_load_2d_hint(gsm + L.w + s * kWStageBytes, &wmap,
+                             static_cast<int>((b0 * kBlkB) >> 4) * 2, static_cast<int>(m0), &w_full[s],
+                             policy_evict_first());
           }
-          total += len[i];
+          __syncwarp();
+        } else {
+          const uint32_t nbytes = static_cast<uint32_t>(i64min(kWChunk / kBlkW, nblk_row - b0) * kBlkB);
+          uint32_t total = 0;
+          uintptr_t lo[4];
+          uint32_t len[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = lane + 32 * i;
+            len[i] = 0;
+            if (m0 + r < a.M) {
+              const uintptr_t src = reinterpret_cast<uintptr_t>(a.W) +
+                                    static_cast<uintptr_t>((m0 + r) * a.rowbytes + b0 * kBlkB);
+              lo[i] = src & ~static_cast<uintptr_t>(15);
+              len[i] = static_cast<uint32_t>(((src + nbytes + 15) & ~static_cast<uintptr_t>(15)) - lo[i]);
+            }
+            total += len[i];
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xFFFFFFFFu, total, o);
+          if (lane == 0) mbar_arrive_expect_tx(&w_full[s], total);
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (len[i])
+              bulk_g2s(gsm + L.w + s * kWStageBytes + (lane + 32 * i) * kWPitch,
+                       reinterpret_cast<const void*>(lo[i]), len[i], &w_full[s], policy_evict_first());
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xFFFFFFFFu, total, o);
-        if (lane == 0) mbar_arrive_expect_tx(&w_full[s], total);
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (len[i])
-            bulk_g2s(gsm + L.w + s * kWStageBytes + (lane + 32 * i) * kWPitch,
-                     reinterpret_cast<const void*>(lo[i]), len[i], &w_full[s], policy_evict_first());
         w_issued = c + 1;
       }
       const int sx = ks % kXStages;
@@ -478,7 +494,25 @@ gq_status gemm_entry(const void* W, int64_t M, int64_t K, const void* X, int xt,
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return GQ_ERR_CUDA;
 
+  // W as rows of 8-byte elements when rows are whole 16-byte granules: a W
+  // stage is then one box of 38 elements (304 bytes) x 128 rows, already at
+  // the row pitch the dequant warps read
+  const int64_t rowbytes = K / kBlkW * kBlkB;
+  const bool w_tma = (rowbytes % 16 == 0) && rowbytes >= kWPitch && M >= kBM;
+  CUtensorMap wmap = {};
+  if (w_tma) {
+    const cuuint64_t wdim[2] = {static_cast<cuuint64_t>(rowbytes / 8), static_cast<cuuint64_t>(M)};
+    const cuuint64_t wstride[1] = {static_cast<cuuint64_t>(rowbytes)};
+    const cuuint32_t wbox[2] = {static_cast<cuuint32_t>(kWPitch / 8), static_cast<cuuint32_t>(kBM)};
+    const cuuint32_t westride[2] = {1, 1};
+    if (enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<void*>(W), wdim, wstride, wbox,
+            westride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return GQ_ERR_CUDA;
+  }
+
   GemmArgs a;
+  a.w_tma = w_tma ? 1 : 0;
   a.W = static_cast<const uint8_t*>(W);
   a.M = M;
   a.K = K;
@@ -508,7 +542,7 @@ gq_status gemm_entry(const void* W, int64_t M, int64_t K, const void* X, int xt,
   }
   const int64_t grid = (M + kBM - 1) / kBM;
   return launch(gemm_kernel<FMT>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem,
-                as_stream(stream), false, xmap, a);
+                as_stream(stream), false, xmap, wmap, a);
 }
 
 }  // namespace
