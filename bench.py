@@ -41,8 +41,8 @@ FALLBACK_HBM_GBS = 6650.0
 GEMV_TRAFFIC = {
     "bytes": 25407744,
     "sources": {
-        "bit_gemv_q4_b200/csrc/gq_gemv.cu": "c19aaf85ea5b879f2aaa30d2c6800b507f4e560801bb17aa0357e490d98e7537",
-        "bit_gemv_q4_b200/csrc/gq_device.cuh": "a2e2779ecb02fd76d9cd3c26065670d43d3cf6839efcb7fd46da6bc987ddcffd",
+        "bit_gemv_q4_b200/csrc/gq_gemv.cu": "3a396a231f0b52d94bea082f9ba47776c70c402d1dd37454c481e99a3489e87c",
+        "bit_gemv_q4_b200/csrc/gq_device.cuh": "c88e136b756c0355212db717041e37b38523df1a913fe4fa63cd047c2a12e5f4",
     },
 }
 
