@@ -250,7 +250,7 @@ def _gemm(name: str, fmt: int, W: torch.Tensor, M: int, K: int, X: torch.Tensor,
         out = torch.empty((B, M), dtype=y_dtype, device=X2.device)
     need = gq_gemm_workspace_bytes(fmt, M, K, B)
     if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=X2.device)
+        workspace = torch.zeros(need, dtype=torch.uint8, device=X2.device)
     ws_bytes = workspace.numel() if workspace is not None else 0
     _check(getattr(lib, name)(_ptr(W), int(M), int(K), _ptr(X2), _DTYPE_CODE[X2.dtype], B,
                               _ptr(out), _DTYPE_CODE[out.dtype], _ptr(workspace), ws_bytes,

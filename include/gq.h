@@ -209,8 +209,16 @@ GQ_API gq_status gq_selftest_gemv_timeout(const void* W, int64_t M, int64_t K, c
  * exactly into two bfloat16 parts, both multiplied by X on the tensor core
  * into one fp32 accumulator, so every product is exact and only the fp32
  * accumulation rounds.
- * workspace / ws_bytes: caller-owned scratch of at least
- * gq_gemm_workspace_bytes(...) bytes (may be NULL when that is 0).
+ * Work split: the 128-row tiles x 64-wide k-steps are divided evenly over
+ * the SMs (stream-K); a tile shared by two or three SMs is combined through
+ * fp32 partial sums, in a fixed order, so results do not depend on
+ * scheduling.
+ * workspace / ws_bytes: caller-owned device scratch of at least
+ * gq_gemm_workspace_bytes(...) bytes (GQ_ERR_WORKSPACE otherwise),
+ * 256-byte aligned, all zero before its first use; a successful call leaves
+ * it ready for the next call of the same or a smaller shape; after a call
+ * that fails or reports GQ_DEV_TIMEOUT, zero it again.  Calls that may run
+ * at the same time need separate workspaces.
  * dev_status: optional, receives GQ_DEV_TIMEOUT if a pipeline wait gives up. */
 GQ_API size_t gq_gemm_workspace_bytes(int fmt, int64_t M, int64_t K, int64_t B);
 GQ_API gq_status gq_gemm_q4_0(const void* W, int64_t M, int64_t K,

@@ -139,7 +139,16 @@ def test_gemm_validation(name, block):
     assert call(W=A + 2) == ALIGN
     assert call(X=A + 8) == ALIGN
     assert call(st=A + 1) == ALIGN
-    assert gq.gq_gemm_workspace_bytes(0, 11008, 4096, 256) >= 0
+    # a valid call without (or with too small) a workspace is refused before
+    # any launch
+    assert call() == 9
+    need = gq.gq_gemm_workspace_bytes(0, 128, K, 16)
+    assert need > 0
+    assert call(ws=A, wsb=need - 1) == 9
+    assert call(ws=A + 16, wsb=need) == ALIGN
+    # counts of the 86 tiles, then two 128 x 256 fp32 parts per SM
+    big = gq.gq_gemm_workspace_bytes(0, 11008, 4096, 256)
+    assert big >= 2 * 128 * 256 * 4 and big % 256 == 0
 
 
 def test_gemv_workspace_sizes_and_checks():

@@ -80,3 +80,41 @@ def test_gemm_matches_gemv_small_batch():
     Yr, bound = oracle.gemm(Q40, q, M, K, *x_for_oracle(X))
     assert_product_close(y1, Yr, bound)
     assert_product_close(y2, Yr, bound)
+
+
+def test_gemm_stream_k_deterministic_and_reusable():
+    # 1000 x 4096 with 36 k-steps per tile spread over every SM: most tiles
+    # are cut between CTAs; their parts are summed in CTA order, so repeated
+    # calls on one workspace give identical bits
+    M, K, B = 1000, 4096, 40
+    q = packed(Q40, M, K)
+    X = synth.activations(B, K, seed=9, dtype=torch.bfloat16).cuda()
+    Wt = torch.from_numpy(q).cuda()
+    ws = torch.zeros(gq.gq_gemm_workspace_bytes(Q40, M, K, B), dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(3):
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        outs.append(gq.gq_gemm_q4_0(Wt, M, K, X, workspace=ws, dev_status=st))
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+    assert torch.equal(outs[0].view(torch.int32), outs[1].view(torch.int32))
+    assert torch.equal(outs[0].view(torch.int32), outs[2].view(torch.int32))
+    Yr, bound = oracle.gemm(Q40, q, M, K, *x_for_oracle(X))
+    assert_product_close(outs[0], Yr, bound)
+
+
+@pytest.mark.parametrize("M,K,B", [(20000, 64, 16), (8192, 256, 16), (3000, 1024, 256)])
+def test_gemm_split_shapes(M, K, B):
+    # one k-step per tile (whole tiles only), short rows with cuts inside
+    # tiles, and the widest batch; checked on rows spanning every tile
+    rows = np.unique(np.concatenate([np.arange(0, M, 29), [M - 1]])).astype(np.int64)
+    check(Q40, M, K, B, rows=rows)
+
+
+def test_gemm_refuses_short_workspace():
+    M, K, B = 256, 512, 16
+    Wt = torch.from_numpy(packed(Q40, M, K)).cuda()
+    X = torch.zeros((B, K), dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(gq.gq_gemm_workspace_bytes(Q40, M, K, B) - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(gq.GQError):
+        gq.gq_gemm_q4_0(Wt, M, K, X, workspace=ws)
