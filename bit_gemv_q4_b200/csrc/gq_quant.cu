@@ -24,21 +24,43 @@ namespace {
 
 constexpr int kQThreads = 256;
 
-// clamp(rint(v / d) + 8, 0, 15) with an IEEE quotient and round-half-even;
-// a zero scale or a non-finite quotient gives code 8.
-__device__ __forceinline__ uint32_t code_of(float v, float d) {
-  if (d == 0.0f) return 8u;
-  const float t = __fdiv_rn(v, d);
-  if (!(fabsf(t) < 1e9f)) return 8u;
-  const int c = __float2int_rn(t) + 8;
-  return static_cast<uint32_t>(min(max(c, 0), 15));
+// Four codes clamp(rint(fl32(v / d)) + 8, 0, 15) as four nibbles (first value
+// in bits 0-3), with the IEEE quotient and round-half-even; a zero, infinite
+// or NaN scale gives code 8.
+//
+// The quotient needs no divide per value: with r = RN(1/d) (one IEEE
+// reciprocal per block), q = RN(v * r) is within one ulp of v/d, e = v - d*q
+// is exact as an FMA, and RN(q + e * r) is the correctly rounded quotient
+// (Markstein's theorem for division with a fused multiply-add: Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990; Muller et al., Handbook of
+// Floating-Point Arithmetic, the chapter on division and square root with an
+// FMA), provided nothing underflows or overflows.  Here d is the block's own
+// scale (absmax/7 rounded to FP16, or S * q_j within a factor 1.5 of it), so
+// |v/d| <= 10.5 and nothing overflows; a quotient small enough to underflow
+// is far from +-0.5 and its code is 8 whatever its last bits.  rint is
+// an add of 1.5 * 2^23, exact and round-half-even for |t| < 2^22.
+__device__ __forceinline__ uint32_t codes4(float4 v, float d, float r) {
+  const bool special = !(d > 0.0f && d < INFINITY);
+  const float2 r2 = make_float2(r, r), nd2 = make_float2(-d, -d);
+  const float2 magic = make_float2(12582912.0f, 12582912.0f);
+  const float2 v01 = make_float2(v.x, v.y), v23 = make_float2(v.z, v.w);
+  float2 q01 = __fmul2_rn(v01, r2), q23 = __fmul2_rn(v23, r2);
+  const float2 e01 = __ffma2_rn(q01, nd2, v01), e23 = __ffma2_rn(q23, nd2, v23);
+  q01 = __fadd2_rn(__ffma2_rn(e01, r2, q01), magic);
+  q23 = __fadd2_rn(__ffma2_rn(e23, r2, q23), magic);
+  // bits(1.5 * 2^23 + k) = 0x4B400000 + k for |k| < 2^22
+  const int bias = static_cast<int>(0x4B400000u) - 8;
+  const int c[4] = {__float_as_int(q01.x) - bias, __float_as_int(q01.y) - bias,
+                    __float_as_int(q23.x) - bias, __float_as_int(q23.y) - bias};
+  uint32_t out = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) out |= static_cast<uint32_t>(min(max(c[i], 0), 15)) << (4 * i);
+  return special ? 0x8888u : out;
 }
 
-// Four codes as four nibbles (first value in bits 0-3).
-__device__ __forceinline__ uint32_t codes4(float4 v, float d) {
-  return code_of(v.x, d) | (code_of(v.y, d) << 4) | (code_of(v.z, d) << 8) |
-         (code_of(v.w, d) << 12);
-}
+// The reciprocal the codes of a block use (any value for a special scale).
+__device__ __forceinline__ float recip_of(float d) { return __frcp_rn(d); }
 
 // Spread four nibbles into the low nibbles of four bytes.
 __device__ __forceinline__ uint32_t spread4(uint32_t a) {
@@ -108,7 +130,7 @@ __global__ void __launch_bounds__(kQThreads)
       const __half dh = __float2half_rn(__fdiv_rn(a, 7.0f));
       const float d = __half2float(dh);
       if (__hisinf(dh)) flags |= GQ_DEV_RANGE;
-      const uint32_t c = codes4(v, d);
+      const uint32_t c = codes4(v, d, recip_of(d));
       const uint32_t partner = __shfl_xor_sync(0xFFFFFFFFu, c, 4);
       if (bl < nb) {
         uint8_t* blk = stage + bl * 18;
@@ -166,7 +188,7 @@ __global__ void __launch_bounds__(kQThreads)
     // codes against the scale the decoder rebuilds, S * q_j
     const float st0 = __fmul_rn(S, static_cast<float>(q0));
     const float st1 = __fmul_rn(S, static_cast<float>(q1));
-    const uint32_t c0 = codes4(v0, st0), c1 = codes4(v1, st1);
+    const uint32_t c0 = codes4(v0, st0, recip_of(st0)), c1 = codes4(v1, st1, recip_of(st1));
     const uint32_t p0 = __shfl_xor_sync(0xFFFFFFFFu, c0, 4);
     const uint32_t p1 = __shfl_xor_sync(0xFFFFFFFFu, c1, 4);
     if (warp < ns) {

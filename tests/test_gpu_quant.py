@@ -147,3 +147,57 @@ def test_quantize_1e9_sampled(fmt):
     assert_bytes_equal(got.ravel(), want, blk_b)
     del w, q
     torch.cuda.empty_cache()
+
+
+def _boundary_values(rng, step, limit, n):
+    """n fp32 values on and one or two ulps around (k + 1/2) * step, |v| <= limit."""
+    ks = rng.integers(-8, 8, size=n)
+    base = ((ks + 0.5) * np.float64(step)).astype(np.float32)
+    nudge = rng.integers(-2, 3, size=n)
+    v = base.copy()
+    for i in range(n):
+        for _ in range(abs(int(nudge[i]))):
+            v[i] = np.nextafter(v[i], np.float32(np.inf if nudge[i] > 0 else -np.inf))
+    return np.where(np.abs(v) <= limit, v, np.float32(0.0)).astype(np.float32)
+
+
+def test_q4_0_codes_at_rounding_boundaries():
+    # every block: one element fixes absmax (so d = FP16(absmax / 7)), the
+    # others sit exactly on a half-way point (k + 1/2) * d -- ties go to even
+    # -- or one or two ulps from it; scales from FP16-subnormal to large
+    rng = np.random.default_rng(2024)
+    nb = 20000
+    absmax = (2.0 ** rng.uniform(-26, 14, size=nb)).astype(np.float32)
+    d = oracle.f16_bits_to_f32(oracle.f32_to_f16_bits(absmax / np.float32(7.0)))
+    x = np.empty((nb, 32), dtype=np.float32)
+    for b in range(nb):
+        x[b] = _boundary_values(rng, d[b], absmax[b], 32)
+        x[b, rng.integers(0, 32)] = absmax[b] * (1 if rng.random() < 0.5 else -1)
+    want, _ = oracle.quantize(Q40, x.ravel())
+    got, st = gpu_quantize(Q40, torch.from_numpy(x))
+    assert st == 0
+    assert_bytes_equal(got, want, 18)
+
+
+def test_ksb_codes_at_rounding_boundaries():
+    # each sub-block's absmax is 7 * d_j, so its FP16 scale is exactly d_j;
+    # the other values sit on and around half-way points of the rebuilt
+    # scale S * q_j that the codes are taken against
+    rng = np.random.default_rng(7)
+    nsb = 2500
+    x = np.empty((nsb, 256), dtype=np.float32)
+    for s in range(nsb):
+        e = rng.uniform(-20, 10)
+        d = oracle.f16_bits_to_f32(oracle.f32_to_f16_bits(
+            (2.0 ** (e + rng.uniform(-3, 0, size=8))).astype(np.float32)))
+        s_bits, q = oracle.ksb_scale_step(oracle.f32_to_f16_bits(d))
+        S = oracle.f16_bits_to_f32(np.array([s_bits], np.uint16))[0]
+        for j in range(8):
+            st = np.float32(S) * np.float32(q[j])
+            limit = np.float32(7.0) * d[j]
+            x[s, 32 * j:32 * (j + 1)] = _boundary_values(rng, st if st > 0 else d[j], limit, 32)
+            x[s, 32 * j + rng.integers(0, 32)] = limit
+    want, _ = oracle.quantize(KSB, x.ravel())
+    got, st = gpu_quantize(KSB, torch.from_numpy(x))
+    assert st == 0
+    assert_bytes_equal(got, want, 138)
