@@ -7,10 +7,12 @@
 //   to INT8 against one FP16 super-scale S = max/127; 2 + 8 + 128 bytes.
 //
 // Both directions are HBM-bound streams (4 B of fp32 per weight against
-// 0.5625 / 0.539 B packed).  Loads are 128-bit and coalesced; a CTA builds
-// the packed bytes of 64 Q4_0 blocks (1152 B) or 8 super-blocks (1104 B) in
-// shared memory and writes them with 16-byte stores.  Block absmax values are
-// warp-shuffle reductions over the 8 lanes that hold one 32-weight block.
+// 0.5625 / 0.539 B packed).  Loads are 128-bit and coalesced; a quantizer CTA
+// builds the packed bytes of 128 Q4_0 blocks (2304 B) or 16 super-blocks
+// (2208 B) in shared memory and writes them with 16-byte stores.  Four lanes
+// hold one 32-weight block; its absmax is a shuffle reduction over them.  The
+// quantizers run near the SM issue rate as much as the HBM rate, so the
+// per-weight work avoids divides and per-code branches (below).
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -24,68 +26,85 @@ namespace {
 
 constexpr int kQThreads = 256;
 
-// Four codes clamp(rint(fl32(v / d)) + 8, 0, 15) as four nibbles (first value
-// in bits 0-3), with the IEEE quotient and round-half-even; a zero, infinite
-// or NaN scale gives code 8.
-//
-// The quotient needs no divide per value: with r = RN(1/d) (one IEEE
-// reciprocal per block), q = RN(v * r) is within one ulp of v/d, e = v - d*q
-// is exact as an FMA, and RN(q + e * r) is the correctly rounded quotient
-// (Markstein's theorem for division with a fused multiply-add: Markstein,
+// Division without a divide.  Every divisor here has a short significand:
+// the FP16 scales (11 bits), S * q_j (at most 18 bits), 7 and 127.  With
+// rb = RN(1/b), q = RN(a * rb) is within 1.5 ulp of a/b, the residual
+// a - q*b comes from one FMA, and RN(q + (a - q*b) * rb) is the correctly
+// rounded quotient.  This is Markstein's FMA division step (Markstein,
 // "Computation of elementary functions on the IBM RISC System/6000
 // processor", IBM J. Res. Dev. 34(1), 1990; Muller et al., Handbook of
-// Floating-Point Arithmetic, the chapter on division and square root with an
-// FMA), provided nothing underflows or overflows.  Here d is the block's own
-// scale (absmax/7 rounded to FP16, or S * q_j within a factor 1.5 of it), so
-// |v/d| <= 10.5 and nothing overflows; a quotient small enough to underflow
-// is far from +-0.5 and its code is 8 whatever its last bits.  rint is
-// an add of 1.5 * 2^23, exact and round-half-even for |t| < 2^22.
-__device__ __forceinline__ uint32_t codes4(float4 v, float d, float r) {
+// Floating-Point Arithmetic, the chapter on division with an FMA); the short
+// divisor is what makes one step enough:
+//   * the exact value of the corrected sum differs from a/b by at most
+//     (1.5 ulp) * 2^-24 from rb and the same again if the residual rounds,
+//     under 2^-22 ulp;
+//   * a/b is never a midpoint between floats (a 24-bit a over a b of p bits
+//     cannot equal a 25-bit odd significand), and a/b - m for a midpoint m is
+//     a nonzero multiple of 2^(e_m - 24 - p) divided by b, at least
+//     2^-(p+1) ulp = 2^-19 ulp for p = 18;
+//   so the final rounding sees a/b's own side of every midpoint.  Operands
+// are finite, a >= 0 or of either sign with |a/b| bounded, b > 0 normal; a
+// quotient that underflows fp32 is below every FP16 and code threshold and
+// its last bits never matter.
+__device__ __forceinline__ float div_short(float a, float b, float rb) {
+  const float q = __fmul_rn(a, rb);
+  return __fmaf_rn(__fmaf_rn(-q, b, a), rb, q);
+}
+
+// FP16(fl32(a / 7)) and FP16(fl32(a / 127)) for maxima a >= 0; a = +inf or
+// NaN (a block of NaNs only) passes through as the IEEE quotient would.
+constexpr float kInv7 = 1.0f / 7.0f;
+constexpr float kInv127 = 1.0f / 127.0f;
+__device__ __forceinline__ __half scale_over(float a, float b, float rb) {
+  return __float2half_rn(a < INFINITY ? div_short(a, b, rb) : a);
+}
+
+// Two codes clamp(rint(fl32(v / d)) + 8, 0, 15) as the halves of an s16x2,
+// the quotient correctly rounded (div_short's argument, with r = RN(1/d)) and
+// rint half to even.  d is the block's own scale (absmax/7 in FP16, or
+// S * q_j within a factor 1.5 of it), so |v/d| <= 16: adding 1.5 * 2^23 + 8
+// rounds to an integer exactly and half-even (8 is even), and the low 16 bits
+// of the sum's encoding are rint(v/d) + 8 as a signed 16-bit value.  A NaN v
+// gives some code in range (its block is reported non-finite).
+__device__ __forceinline__ uint32_t code_pair(float a, float b, float d, float r) {
+  const float2 v = make_float2(a, b), r2 = make_float2(r, r);
+  float2 q = __fmul2_rn(v, r2);
+  const float2 e = __ffma2_rn(q, make_float2(-d, -d), v);
+  q = __fadd2_rn(__ffma2_rn(e, r2, q), make_float2(12582920.0f, 12582920.0f));
+  const uint32_t k = __byte_perm(__float_as_uint(q.x), __float_as_uint(q.y), 0x5410);
+  return __vimin_s16x2_relu(k, 0x000F000Fu);  // max(min(k, 15), 0) per half
+}
+
+// The four qs bytes of one lane: byte i = code(lo[i]) | code(hi[i]) << 4, the
+// lo/hi split of the Q4_0 chapter, section 4.2.1 (lo holds weights 4t..4t+3,
+// hi weights 16+4t..19+4t).  A zero, infinite or NaN scale gives code 8.
+__device__ __forceinline__ uint32_t qs_bytes(float4 lo, float4 hi, float d) {
+  const float r = __frcp_rn(d);
+  const uint32_t b01 = code_pair(lo.x, lo.y, d, r) | (code_pair(hi.x, hi.y, d, r) << 4);
+  const uint32_t b23 = code_pair(lo.z, lo.w, d, r) | (code_pair(hi.z, hi.w, d, r) << 4);
   const bool special = !(d > 0.0f && d < INFINITY);
-  const float2 r2 = make_float2(r, r), nd2 = make_float2(-d, -d);
-  const float2 magic = make_float2(12582912.0f, 12582912.0f);
-  const float2 v01 = make_float2(v.x, v.y), v23 = make_float2(v.z, v.w);
-  float2 q01 = __fmul2_rn(v01, r2), q23 = __fmul2_rn(v23, r2);
-  const float2 e01 = __ffma2_rn(q01, nd2, v01), e23 = __ffma2_rn(q23, nd2, v23);
-  q01 = __fadd2_rn(__ffma2_rn(e01, r2, q01), magic);
-  q23 = __fadd2_rn(__ffma2_rn(e23, r2, q23), magic);
-  // bits(1.5 * 2^23 + k) = 0x4B400000 + k for |k| < 2^22
-  const int bias = static_cast<int>(0x4B400000u) - 8;
-  const int c[4] = {__float_as_int(q01.x) - bias, __float_as_int(q01.y) - bias,
-                    __float_as_int(q23.x) - bias, __float_as_int(q23.y) - bias};
-  uint32_t out = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) out |= static_cast<uint32_t>(min(max(c[i], 0), 15)) << (4 * i);
-  return special ? 0x8888u : out;
+  return special ? 0x88888888u : __byte_perm(b01, b23, 0x6420);
 }
 
-// The reciprocal the codes of a block use (any value for a special scale).
-__device__ __forceinline__ float recip_of(float d) { return __frcp_rn(d); }
-
-// Spread four nibbles into the low nibbles of four bytes.
-__device__ __forceinline__ uint32_t spread4(uint32_t a) {
-  return (a & 0xFu) | ((a & 0xF0u) << 4) | ((a & 0xF00u) << 8) | ((a & 0xF000u) << 12);
+// max |v| over a lane's eight values with NaN propagation (NaN if any value
+// is NaN, else +inf if any is infinite), so one compare finds a non-finite
+// input.  The xorsign form takes absolute values of its operands; the sign it
+// leaves is dropped at the end.
+__device__ __forceinline__ float amax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.xorsign.abs.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float absmax8(float4 u, float4 v) {
+  const float a = amax_nan(amax_nan(u.x, u.y), amax_nan(u.z, u.w));
+  const float b = amax_nan(amax_nan(v.x, v.y), amax_nan(v.z, v.w));
+  return fabsf(amax_nan(a, b));
 }
 
-// qs bytes for weights j..j+3 (low nibbles, from `lo`) and j+16..j+19 (high
-// nibbles, from `hi`): the lo/hi split of the Q4_0 chapter, section 4.2.1.
-__device__ __forceinline__ uint32_t pack_lohi(uint32_t lo, uint32_t hi) {
-  return spread4(lo) | (spread4(hi) << 4);
-}
-
-__device__ __forceinline__ float absmax4(float4 v) {
-  return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-}
-
-__device__ __forceinline__ bool finite4(float4 v) {
-  return isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
-}
-
-// max over the 8 lanes of an aligned group of 8
-__device__ __forceinline__ float group8_max(float a) {
+// max over the 4 lanes of an aligned group of 4
+__device__ __forceinline__ float group4_max(float a) {
   a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
   a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
-  a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 4));
   return a;
 }
 
@@ -108,109 +127,140 @@ __device__ __forceinline__ void flush_tile(uint8_t* dst, const uint8_t* stage, i
 }
 
 // ---------------------------------------------------------------- Q4_0 quantize
-// CTA tile: 64 blocks (2048 floats).  Warp w owns blocks 8w..8w+7; in each of
-// two passes its lanes hold 4 blocks, 8 lanes (one float4 each) per block.
+// CTA tile: 128 blocks (4096 floats).  Four lanes share a block: lane t of a
+// block holds weights 4t..4t+3 and 16+4t..19+4t, the two halves whose codes
+// fill qs bytes 4t..4t+3, so a lane packs its bytes without a partner.  Warp w
+// owns blocks 16w..16w+15, eight per pass.  A CTA walks its tiles with the
+// next tile's loads issued before the current tile is packed, so each lane
+// keeps 64 B of reads in flight while it computes.
+constexpr int kQ0Tile = 128;
+
 __global__ void __launch_bounds__(kQThreads)
     quantize_q4_0_kernel(const float* __restrict__ x, int64_t nblk, uint8_t* __restrict__ out,
                          int* dev_status) {
-  __shared__ __align__(16) uint8_t stage[64 * 18];
+  __shared__ __align__(16) uint8_t stage[kQ0Tile * 18];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 3, sub = lane & 7;
+  const int t = lane & 3;
   int flags = 0;
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * 64; base < nblk;
-       base += static_cast<int64_t>(gridDim.x) * 64) {
-    const int nb = static_cast<int>(i64min(64, nblk - base));
+  const int64_t step = static_cast<int64_t>(gridDim.x) * kQ0Tile;
+  // this lane's two float4 of pass h of the tile at `b`
+  auto load = [&](int64_t b, float4 (&l)[2], float4 (&u)[2]) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int bl = warp * 8 + h * 4 + g;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (bl < nb) v = __ldcs(reinterpret_cast<const float4*>(x + (base + bl) * 32) + sub);
-      if (!finite4(v)) flags |= GQ_DEV_NONFINITE;
-      const float a = group8_max(absmax4(v));
-      const __half dh = __float2half_rn(__fdiv_rn(a, 7.0f));
+      const int64_t bl = b + warp * 16 + h * 8 + (lane >> 2);
+      l[h] = u[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (bl < nblk) {
+        const float4* src = reinterpret_cast<const float4*>(x + bl * 32);
+        l[h] = __ldcs(src + t);
+        u[h] = __ldcs(src + 4 + t);
+      }
+    }
+  };
+  float4 lo[2], hi[2];
+  load(static_cast<int64_t>(blockIdx.x) * kQ0Tile, lo, hi);
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * kQ0Tile; base < nblk; base += step) {
+    const int nb = static_cast<int>(i64min(kQ0Tile, nblk - base));
+    float4 nlo[2], nhi[2];  // the next tile's values, in flight while this one is packed
+    load(base + step, nlo, nhi);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int bl = warp * 16 + h * 8 + (lane >> 2);
+      const float own = absmax8(lo[h], hi[h]);
+      if (!(own < INFINITY)) flags |= GQ_DEV_NONFINITE;
+      const __half dh = scale_over(group4_max(own), 7.0f, kInv7);
       const float d = __half2float(dh);
       if (__hisinf(dh)) flags |= GQ_DEV_RANGE;
-      const uint32_t c = codes4(v, d, recip_of(d));
-      const uint32_t partner = __shfl_xor_sync(0xFFFFFFFFu, c, 4);
+      const uint32_t b = qs_bytes(lo[h], hi[h], d);
       if (bl < nb) {
         uint8_t* blk = stage + bl * 18;
-        if (sub == 0) st_u16(blk, __half_as_ushort(dh));
-        if (sub < 4) {
-          const uint32_t b = pack_lohi(c, partner);
-          st_u16(blk + 2 + 4 * sub, b & 0xFFFFu);
-          st_u16(blk + 4 + 4 * sub, b >> 16);
-        }
+        if (t == 0) st_u16(blk, __half_as_ushort(dh));
+        st_u16(blk + 2 + 4 * t, b & 0xFFFFu);
+        st_u16(blk + 4 + 4 * t, b >> 16);
       }
     }
     __syncthreads();
-    flush_tile(out + base * 18, stage, nb * 18, 64 * 18);
+    flush_tile(out + base * 18, stage, nb * 18, kQ0Tile * 18);
     __syncthreads();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      lo[h] = nlo[h];
+      hi[h] = nhi[h];
+    }
   }
   if (flags) report(dev_status, flags);
 }
 
 // ----------------------------------------------------------------- ksb quantize
-// CTA tile: 8 super-blocks; warp w owns super-block w.  Lane l holds float4 l
-// (sub-block l/8) and float4 32+l (sub-block 4+l/8).
+// CTA tile: 16 super-blocks; warp w owns super-blocks w and 8 + w, one per
+// pass, with the next tile's loads in flight as in the Q4_0 kernel.  Lane 4j + t holds, of sub-block j,
+// weights 4t..4t+3 and 16+4t..19+4t (the Q4_0 lane split of one block).
+constexpr int kKsbTile = 16;
+
 __global__ void __launch_bounds__(kQThreads)
     quantize_ksb_kernel(const float* __restrict__ x, int64_t nsb, uint8_t* __restrict__ out,
                         int* dev_status) {
-  __shared__ __align__(16) uint8_t stage[8 * 138];
+  __shared__ __align__(16) uint8_t stage[kKsbTile * 138];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 3, sub = lane & 7;
+  const int j = lane >> 2, t = lane & 3;
   int flags = 0;
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * 8; base < nsb;
-       base += static_cast<int64_t>(gridDim.x) * 8) {
-    const int ns = static_cast<int>(i64min(8, nsb - base));
-    float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
-    if (warp < ns) {
-      const float4* p = reinterpret_cast<const float4*>(x + (base + warp) * 256);
-      v0 = __ldcs(p + lane);
-      v1 = __ldcs(p + 32 + lane);
-    }
-    if (!finite4(v0) || !finite4(v1)) flags |= GQ_DEV_NONFINITE;
-    // each sub-block's own FP16 scale, absmax / 7
-    const __half d0h = __float2half_rn(__fdiv_rn(group8_max(absmax4(v0)), 7.0f));
-    const __half d1h = __float2half_rn(__fdiv_rn(group8_max(absmax4(v1)), 7.0f));
-    if (__hisinf(d0h) || __hisinf(d1h)) flags |= GQ_DEV_RANGE;
-    const float d0 = __half2float(d0h), d1 = __half2float(d1h);
-    // super-scale S = FP16(max_j d_j / 127)
-    float m = fmaxf(d0, d1);
-    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 8));
-    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
-    const __half sh = __float2half_rn(__fdiv_rn(m, 127.0f));
-    const float S = __half2float(sh);
-    int q0 = 0, q1 = 0;
-    if (S != 0.0f && !__hisinf(sh)) {
-      q0 = min(max(__float2int_rn(__fdiv_rn(d0, S)), 0), 127);
-      q1 = min(max(__float2int_rn(__fdiv_rn(d1, S)), 0), 127);
-    }
-    // codes against the scale the decoder rebuilds, S * q_j
-    const float st0 = __fmul_rn(S, static_cast<float>(q0));
-    const float st1 = __fmul_rn(S, static_cast<float>(q1));
-    const uint32_t c0 = codes4(v0, st0, recip_of(st0)), c1 = codes4(v1, st1, recip_of(st1));
-    const uint32_t p0 = __shfl_xor_sync(0xFFFFFFFFu, c0, 4);
-    const uint32_t p1 = __shfl_xor_sync(0xFFFFFFFFu, c1, 4);
-    if (warp < ns) {
-      uint8_t* sb = stage + warp * 138;
-      if (lane == 0) st_u16(sb, __half_as_ushort(sh));
-      if (sub == 0) {
-        sb[2 + g] = static_cast<uint8_t>(q0);
-        sb[6 + g] = static_cast<uint8_t>(q1);
+  const int64_t step = static_cast<int64_t>(gridDim.x) * kKsbTile;
+  auto load = [&](int64_t b, float4 (&l)[2], float4 (&u)[2]) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int64_t sb = b + warp + 8 * h;
+      l[h] = u[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (sb < nsb) {
+        const float4* src = reinterpret_cast<const float4*>(x + sb * 256 + 32 * j);
+        l[h] = __ldcs(src + t);
+        u[h] = __ldcs(src + 4 + t);
       }
-      if (sub < 4) {
-        const uint32_t b0 = pack_lohi(c0, p0), b1 = pack_lohi(c1, p1);
-        uint8_t* s0 = sb + 10 + 16 * g + 4 * sub;
-        uint8_t* s1 = sb + 10 + 16 * (4 + g) + 4 * sub;
-        st_u16(s0, b0 & 0xFFFFu);
-        st_u16(s0 + 2, b0 >> 16);
-        st_u16(s1, b1 & 0xFFFFu);
-        st_u16(s1 + 2, b1 >> 16);
+    }
+  };
+  float4 lo[2], hi[2];
+  load(static_cast<int64_t>(blockIdx.x) * kKsbTile, lo, hi);
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * kKsbTile; base < nsb; base += step) {
+    const int ns = static_cast<int>(i64min(kKsbTile, nsb - base));
+    float4 nlo[2], nhi[2];  // the next tile's values, in flight while this one is packed
+    load(base + step, nlo, nhi);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int sb = warp + 8 * h;
+      const float own = absmax8(lo[h], hi[h]);
+      if (!(own < INFINITY)) flags |= GQ_DEV_NONFINITE;
+      // the sub-block's own FP16 scale, absmax / 7
+      const __half dh = scale_over(group4_max(own), 7.0f, kInv7);
+      if (__hisinf(dh)) flags |= GQ_DEV_RANGE;
+      const float d = __half2float(dh);
+      // super-scale S = FP16(max_j d_j / 127)
+      float m = d;
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 8));
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
+      const __half sh = scale_over(m, 127.0f, kInv127);
+      const float S = __half2float(sh);
+      int q = 0;
+      if (S != 0.0f && !__hisinf(sh))
+        q = min(max(__float2int_rn(div_short(d, S, __frcp_rn(S))), 0), 127);
+      // codes against the scale the decoder rebuilds, S * q_j
+      const float st = __fmul_rn(S, static_cast<float>(q));
+      const uint32_t b = qs_bytes(lo[h], hi[h], st);
+      if (sb < ns) {
+        uint8_t* blk = stage + sb * 138;
+        if (lane == 0) st_u16(blk, __half_as_ushort(sh));
+        if (t == 0) blk[2 + j] = static_cast<uint8_t>(q);
+        uint8_t* qs = blk + 10 + 16 * j + 4 * t;
+        st_u16(qs, b & 0xFFFFu);
+        st_u16(qs + 2, b >> 16);
       }
     }
     __syncthreads();
-    flush_tile(out + base * 138, stage, ns * 138, 8 * 138);
+    flush_tile(out + base * 138, stage, ns * 138, kKsbTile * 138);
     __syncthreads();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      lo[h] = nlo[h];
+      hi[h] = nhi[h];
+    }
   }
   if (flags) report(dev_status, flags);
 }
@@ -295,6 +345,20 @@ int stream_grid(int64_t tiles) {
   return static_cast<int>(tiles < cap ? (tiles > 0 ? tiles : 1) : cap);
 }
 
+// One wave of resident CTAs (or fewer when there are fewer tiles): the
+// quantizers prefetch across their own tiles, so a second wave would only
+// add a tail.
+template <typename Kernel>
+int resident_grid(Kernel kernel, int64_t tiles) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kQThreads, 0) !=
+          cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
+  return static_cast<int>(tiles < cap ? (tiles > 0 ? tiles : 1) : cap);
+}
+
 gq_status check_common(const void* in, int64_t n, int block, const void* out, const int* st) {
   if (n < 0) return GQ_ERR_INVALID_ARG;
   if (n % block) return GQ_ERR_SHAPE;
@@ -317,8 +381,9 @@ GQ_API gq_status gq_quantize_q4_0(const float* x, int64_t n, void* out, int* dev
   gq_status s = check_common(x, n, 32, out, dev_status);
   if (s != GQ_OK || n == 0) return s;
   const int64_t nblk = n / 32;
-  return launch(quantize_q4_0_kernel, dim3(stream_grid((nblk + 63) / 64)), dim3(kQThreads), 0,
-                as_stream(stream), false, x, nblk, static_cast<uint8_t*>(out), dev_status);
+  const dim3 grid(resident_grid(quantize_q4_0_kernel, (nblk + kQ0Tile - 1) / kQ0Tile));
+  return launch(quantize_q4_0_kernel, grid, dim3(kQThreads), 0, as_stream(stream), false, x, nblk,
+                static_cast<uint8_t*>(out), dev_status);
 }
 
 GQ_API gq_status gq_quantize_ksb(const float* x, int64_t n, void* out, int* dev_status,
@@ -326,8 +391,9 @@ GQ_API gq_status gq_quantize_ksb(const float* x, int64_t n, void* out, int* dev_
   gq_status s = check_common(x, n, 256, out, dev_status);
   if (s != GQ_OK || n == 0) return s;
   const int64_t nsb = n / 256;
-  return launch(quantize_ksb_kernel, dim3(stream_grid((nsb + 7) / 8)), dim3(kQThreads), 0,
-                as_stream(stream), false, x, nsb, static_cast<uint8_t*>(out), dev_status);
+  const dim3 grid(resident_grid(quantize_ksb_kernel, (nsb + kKsbTile - 1) / kKsbTile));
+  return launch(quantize_ksb_kernel, grid, dim3(kQThreads), 0, as_stream(stream), false, x, nsb,
+                static_cast<uint8_t*>(out), dev_status);
 }
 
 GQ_API gq_status gq_dequantize_q4_0(const void* q, int64_t n, float* out, void* stream) {

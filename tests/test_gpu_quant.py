@@ -117,10 +117,20 @@ def test_quantize_status_flags(fmt):
     _, flags = oracle.quantize(fmt, x)
     assert st == flags == gq.GQ_DEV_RANGE
     x[40] = 1.0
-    x[300] = np.nan
+    for bad in (np.nan, np.inf, -np.inf):
+        x[300] = bad
+        _, st = gpu_quantize(fmt, torch.from_numpy(x))
+        assert st & gq.GQ_DEV_NONFINITE
+        assert gq.gq_status_from_dev(st) == 5
+    # a block of NaNs only, and a non-finite value as the last of a tile
+    x[:] = 0.0
+    x[-32:] = np.nan
     _, st = gpu_quantize(fmt, torch.from_numpy(x))
     assert st & gq.GQ_DEV_NONFINITE
-    assert gq.gq_status_from_dev(st) == 5
+    x[:] = 0.0
+    x[-1] = -np.inf
+    _, st = gpu_quantize(fmt, torch.from_numpy(x))
+    assert st & gq.GQ_DEV_NONFINITE
 
 
 @pytest.mark.parametrize("fmt", [Q40, KSB])
@@ -200,4 +210,61 @@ def test_ksb_codes_at_rounding_boundaries():
     want, _ = oracle.quantize(KSB, x.ravel())
     got, st = gpu_quantize(KSB, torch.from_numpy(x))
     assert st == 0
+    assert_bytes_equal(got, want, 138)
+
+
+def _nudge32(v, k):
+    """v moved by k fp32 ulps (elementwise)."""
+    v = v.astype(np.float32).copy()
+    for i in range(v.size):
+        for _ in range(abs(int(k[i]))):
+            v[i] = np.nextafter(v[i], np.float32(np.inf if k[i] > 0 else -np.inf))
+    return v
+
+
+def test_q4_0_scales_at_fp16_midpoints():
+    # absmax = 7 * m for m half-way between two FP16 values (exact in fp32),
+    # then 0-3 fp32 ulps either side: absmax / 7 lands on or next to an FP16
+    # rounding midpoint, so the FP16 scale depends on the last bit of the fp32
+    # quotient; FP16-subnormal scales up to the largest finite one
+    rng = np.random.default_rng(31)
+    nb = 20000
+    h = rng.integers(1, 0x7BFF, size=nb).astype(np.uint16)
+    lo = oracle.f16_bits_to_f32(h).astype(np.float64)
+    hi = oracle.f16_bits_to_f32((h + 1).astype(np.uint16)).astype(np.float64)
+    absmax = _nudge32((7.0 * (lo + hi) / 2.0).astype(np.float32), rng.integers(-3, 4, size=nb))
+    x = (rng.uniform(-0.9, 0.9, size=(nb, 32)) * absmax[:, None]).astype(np.float32)
+    pos = rng.integers(0, 32, size=nb)
+    x[np.arange(nb), pos] = absmax * np.where(rng.random(nb) < 0.5, 1, -1).astype(np.float32)
+    want, flags = oracle.quantize(Q40, x.ravel())
+    got, st = gpu_quantize(Q40, torch.from_numpy(x))
+    assert st == flags == 0
+    assert_bytes_equal(got, want, 18)
+
+
+def test_ksb_subscales_at_half_integers():
+    # the largest sub-block scale is 127 * S0 for S0 of 3 significant bits, so
+    # the super-scale is exactly S0 and S0 * (k + 1/2) is an FP16 value: the
+    # other seven sub-block scales sit on such a tie (rounded half to even
+    # into q_j) or one FP16 ulp either side of it
+    rng = np.random.default_rng(37)
+    nsb = 4000
+    e = rng.integers(-24, 1, size=nsb).astype(np.float64)
+    s0 = (2.0 ** e) * (1.0 + rng.integers(0, 4, size=nsb) / 4.0)
+    dmax = 127.0 * s0
+    x = np.empty((nsb, 256), dtype=np.float32)
+    for s in range(nsb):
+        k = rng.integers(0, 127, size=8)
+        dj = oracle.f32_to_f16_bits((s0[s] * (k + 0.5)).astype(np.float32))
+        dj = np.clip(dj.astype(np.int64) + rng.integers(-1, 2, size=8), 1, 0x7BFF)
+        d = oracle.f16_bits_to_f32(dj.astype(np.uint16)).astype(np.float64)
+        d[0] = dmax[s]
+        d = np.minimum(d, dmax[s])
+        limit = (7.0 * d).astype(np.float32)  # exact: d has at most 11 bits
+        blk = rng.uniform(-0.9, 0.9, size=(8, 32)) * limit[:, None]
+        blk[np.arange(8), rng.integers(0, 32, size=8)] = limit
+        x[s] = blk.astype(np.float32).ravel()
+    want, flags = oracle.quantize(KSB, x.ravel())
+    got, st = gpu_quantize(KSB, torch.from_numpy(x))
+    assert st == flags == 0
     assert_bytes_equal(got, want, 138)
