@@ -192,8 +192,9 @@ __global__ void __launch_bounds__(kQThreads)
 
 // ----------------------------------------------------------------- ksb quantize
 // CTA tile: 16 super-blocks; warp w owns super-blocks w and 8 + w, one per
-// pass, with the next tile's loads in flight as in the Q4_0 kernel.  Lane 4j + t holds, of sub-block j,
-// weights 4t..4t+3 and 16+4t..19+4t (the Q4_0 lane split of one block).
+// pass, with the next tile's loads in flight as in the Q4_0 kernel.  Lane
+// 4j + t holds, of sub-block j, weights 4t..4t+3 and 16+4t..19+4t (the Q4_0
+// lane split of one block).
 constexpr int kKsbTile = 16;
 
 __global__ void __launch_bounds__(kQThreads)
