@@ -73,7 +73,12 @@ constexpr int kStageBytes = kRows * kPitch + 16;    // +16: window-read slack
 constexpr int kStages = GQ_GEMV_STAGES;
 constexpr int kXBlk = 64;                           // B-fragment bytes per 32 weights
 constexpr int kXStride = (kChunkW / 32) * kXBlk + 64;  // per (chunk, batch row), padded
-constexpr int kXSmemMax = 72 * 1024;                // activation window budget
+constexpr int kRedBytes = 2 * kConsumers * 32 * 4 * 4;  // cross-warp reduction
+// activation window budget: what the stages and the reduction leave of the
+// 227 KB a CTA may hold, at most 72 KB
+constexpr int kXSmemFree = 227 * 1024 - kStages * kStageBytes - kRedBytes - 1024;
+constexpr int kXSmemMax = kXSmemFree < 72 * 1024 ? kXSmemFree : 72 * 1024;
+static_assert(kXSmemMax >= 16 * 1024, "pipeline shape");
 static_assert(kChunkW == 1024 || kChunkW == 2048, "supported chunk sizes");
 static_assert(kSubPerWarp % 2 == 0, "blocks per warp come in pairs");
 
@@ -170,9 +175,24 @@ __device__ __forceinline__ uint32_t ld32_even(uint32_t off) {
   return __byte_perm(ld32(b), ld32(b + 4), (off & 2u) ? 0x5432u : 0x3210u);
 }
 
+// The activation fragment of one block.  With one activation vector only B
+// columns 0 and 2 carry it (lane groups 0 and 2 load, every other lane holds
+// zeros): the shared-memory load then touches 2 of the warp's 8 lane
+// quarters, and columns 0 and 2 of the result put row r in lane t = 0 and
+// row r+8 in lane t = 1.
+template <bool NB1>
+__device__ __forceinline__ uint4 x_frag(uint32_t xp) {
+  if constexpr (NB1) {
+    const int lane = threadIdx.x & 31;
+    return (lane & 0x14) == 0 ? ld128(xp) : make_uint4(0u, 0u, 0u, 0u);
+  } else {
+    return ld128(xp);
+  }
+}
+
 // One 32-weight block for rows r (codes qa) and r+8 (codes qb): both k16
 // MMAs over every activation term, into a fresh fragment c.
-template <int XT>
+template <int XT, bool NB1>
 __device__ __forceinline__ void block_mma(float c[4], uint32_t qa, uint32_t qb, uint32_t xp,
                                           uint32_t term_stride) {
   constexpr int kTerms = (XT == XT_F32) ? 3 : 1;
@@ -180,7 +200,7 @@ __device__ __forceinline__ void block_mma(float c[4], uint32_t qa, uint32_t qb, 
   if constexpr (XT == XT_F16) {
     decode_f16(qa, ra);
     decode_f16(qb, rb);
-    const uint4 xv = ld128(xp);
+    const uint4 xv = x_frag<NB1>(xp);
     mma_f16_z(c, ra[0], rb[0], ra[2], rb[2], xv.x, xv.y);
     mma_f16(c, ra[1], rb[1], ra[3], rb[3], xv.z, xv.w);
   } else {
@@ -188,7 +208,7 @@ __device__ __forceinline__ void block_mma(float c[4], uint32_t qa, uint32_t qb, 
     decode_bf16(qb, rb);
 #pragma unroll
     for (int tm = 0; tm < kTerms; ++tm) {
-      const uint4 xv = ld128(xp + tm * term_stride);
+      const uint4 xv = x_frag<NB1>(xp + tm * term_stride);
       if (tm == 0)
         mma_bf16_z(c, ra[0], rb[0], ra[2], rb[2], xv.x, xv.y);
       else
@@ -199,23 +219,29 @@ __device__ __forceinline__ void block_mma(float c[4], uint32_t qa, uint32_t qb, 
 }
 
 // Scale a block's fragment and accumulate: acc[i] += d(row) * c[i].  With one
-// activation vector every column of c holds the same value; only columns 0
-// of rows r and r+8 are kept.
+// activation vector (x_frag) lane t = 0 keeps row r (c[0], column 0) and
+// lane t = 1 row r+8 (c[2], column 2), each in acc[0] with its own row's
+// scale d0; lanes t = 2, 3 accumulate zeros.
 template <bool NB1>
 __device__ __forceinline__ void scale_acc(float acc[4], const float c[4], float d0, float d1) {
-  acc[0] = fmaf(d0, c[0], acc[0]);
-  acc[2] = fmaf(d1, c[2], acc[2]);
-  if constexpr (!NB1) {
+  if constexpr (NB1) {
+    const int t = threadIdx.x & 3;
+    acc[0] = fmaf(d0, (t & 1) ? c[2] : c[0], acc[0]);
+  } else {
+    acc[0] = fmaf(d0, c[0], acc[0]);
+    acc[2] = fmaf(d1, c[2], acc[2]);
     acc[1] = fmaf(d0, c[1], acc[1]);
     acc[3] = fmaf(d1, c[3], acc[3]);
   }
 }
 
 // ---------------------------------------------------------------- Q4_0 body
-// Block j of a stage: its two rows' code words and scales.
-template <bool ALIGNED, int J>
-__device__ __forceinline__ void q40_load(uint32_t row0, uint32_t row1, int t, int jb,
-                                         uint32_t& qa, uint32_t& qb, float& da, float& db) {
+// Block j of a stage: its two rows' code words and scales (with one
+// activation vector only the scale of this lane's output row, at rowd).
+template <bool ALIGNED, int J, bool NB1>
+__device__ __forceinline__ void q40_load(uint32_t row0, uint32_t row1, uint32_t rowd, int t,
+                                         int jb, uint32_t& qa, uint32_t& qb, float& da,
+                                         float& db) {
   const uint32_t a = row0 + jb * 18;
   const uint32_t b = row1 + jb * 18;
   if constexpr (ALIGNED) {
@@ -227,8 +253,13 @@ __device__ __forceinline__ void q40_load(uint32_t row0, uint32_t row1, int t, in
     qa = ld32_even(a + 2 + 4 * t);
     qb = ld32_even(b + 2 + 4 * t);
   }
-  da = half_bits_to_float(ld16(a));
-  db = half_bits_to_float(ld16(b));
+  if constexpr (NB1) {
+    da = half_bits_to_float(ld16(rowd + jb * 18));
+    db = da;
+  } else {
+    da = half_bits_to_float(ld16(a));
+    db = half_bits_to_float(ld16(b));
+  }
 }
 
 // A consumer warp's blocks w*kSubPerWarp .. +kSubPerWarp-1 of one stage.  A
@@ -239,18 +270,20 @@ __device__ __forceinline__ void q40_chunk(float acc[4], uint32_t row0, uint32_t 
                                           uint32_t xw, uint32_t term_stride, int w, int t,
                                           int nvalid) {
   const int jw = w * kSubPerWarp;  // even
+  const uint32_t rowd = (t & 1) ? row1 : row0;
   if (nvalid >= kSubPerWarp) {
     uint32_t qa[kSubPerWarp], qb[kSubPerWarp];
     float da[kSubPerWarp], db[kSubPerWarp];
 #pragma unroll
     for (int j = 0; j < kSubPerWarp; j += 2) {
-      q40_load<ALIGNED, 0>(row0, row1, t, jw + j, qa[j], qb[j], da[j], db[j]);
-      q40_load<ALIGNED, 1>(row0, row1, t, jw + j + 1, qa[j + 1], qb[j + 1], da[j + 1], db[j + 1]);
+      q40_load<ALIGNED, 0, NB1>(row0, row1, rowd, t, jw + j, qa[j], qb[j], da[j], db[j]);
+      q40_load<ALIGNED, 1, NB1>(row0, row1, rowd, t, jw + j + 1, qa[j + 1], qb[j + 1], da[j + 1],
+                                db[j + 1]);
     }
 #pragma unroll
     for (int j = 0; j < kSubPerWarp; ++j) {
       float c[4];
-      block_mma<XT>(c, qa[j], qb[j], xw + (jw + j) * kXBlk, term_stride);
+      block_mma<XT, NB1>(c, qa[j], qb[j], xw + (jw + j) * kXBlk, term_stride);
       scale_acc<NB1>(acc, c, da[j], db[j]);
     }
   } else {
@@ -258,9 +291,9 @@ __device__ __forceinline__ void q40_chunk(float acc[4], uint32_t row0, uint32_t 
     for (int j = 0; j < nvalid; ++j) {
       uint32_t qa, qb;
       float da, db;
-      q40_load<false, 0>(row0, row1, t, jw + j, qa, qb, da, db);
+      q40_load<false, 0, NB1>(row0, row1, rowd, t, jw + j, qa, qb, da, db);
       float c[4];
-      block_mma<XT>(c, qa, qb, xw + (jw + j) * kXBlk, term_stride);
+      block_mma<XT, NB1>(c, qa, qb, xw + (jw + j) * kXBlk, term_stride);
       scale_acc<NB1>(acc, c, da, db);
     }
   }
@@ -276,14 +309,17 @@ __device__ __forceinline__ void ksb_chunk(float acc[4], uint32_t row0, uint32_t 
   const int sb = (w * kSubPerWarp) >> 3, j0 = (w * kSubPerWarp) & 7;
   const uint32_t a = row0 + sb * 138;
   const uint32_t b = row1 + sb * 138;
-  const float Sa = half_bits_to_float(ld16(a));
-  const float Sb = half_bits_to_float(ld16(b));
+  // scales of rows r and r+8; with one activation vector only this lane's
+  // output row (scale_acc), read into both
+  const uint32_t sa = NB1 ? ((t & 1) ? b : a) : a;
+  const float Sa = half_bits_to_float(ld16(sa));
+  const float Sb = NB1 ? Sa : half_bits_to_float(ld16(b));
   uint32_t qja[2], qjb[2];
-  qja[0] = ld32_even(a + 2 + j0);
-  qjb[0] = ld32_even(b + 2 + j0);
+  qja[0] = ld32_even(sa + 2 + j0);
+  qjb[0] = NB1 ? qja[0] : ld32_even(b + 2 + j0);
   if constexpr (kSubPerWarp > 4) {
-    qja[1] = ld32_even(a + 6 + j0);
-    qjb[1] = ld32_even(b + 6 + j0);
+    qja[1] = ld32_even(sa + 6 + j0);
+    qjb[1] = NB1 ? qja[1] : ld32_even(b + 6 + j0);
   }
   float sacc[4] = {0.f, 0.f, 0.f, 0.f};
   constexpr int kBatch = kSubPerWarp < 4 ? kSubPerWarp : 4;
@@ -298,7 +334,7 @@ __device__ __forceinline__ void ksb_chunk(float acc[4], uint32_t row0, uint32_t 
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
       float c[4];
-      block_mma<XT>(c, na[j], nb[j], xw + (8 * sb + j0 + h + j) * kXBlk, term_stride);
+      block_mma<XT, NB1>(c, na[j], nb[j], xw + (8 * sb + j0 + h + j) * kXBlk, term_stride);
       const int q = h + j;  // sub-block index within this warp's share
       const float fa = static_cast<float>(static_cast<int8_t>((qja[q >> 2] >> (8 * (q & 3))) & 0xFFu));
       const float fb = static_cast<float>(static_cast<int8_t>((qjb[q >> 2] >> (8 * (q & 3))) & 0xFFu));
@@ -306,8 +342,8 @@ __device__ __forceinline__ void ksb_chunk(float acc[4], uint32_t row0, uint32_t 
     }
   }
   acc[0] = fmaf(Sa, sacc[0], acc[0]);
-  acc[2] = fmaf(Sb, sacc[2], acc[2]);
   if constexpr (!NB1) {
+    acc[2] = fmaf(Sb, sacc[2], acc[2]);
     acc[1] = fmaf(Sa, sacc[1], acc[1]);
     acc[3] = fmaf(Sb, sacc[3], acc[3]);
   }
@@ -369,8 +405,8 @@ __device__ __forceinline__ void store_x8(uint8_t* xs, const void* xsrc, int B, i
 // Load activations [k_begin, k_end) of all batch rows into shared memory in
 // B-fragment order: for each 32 weights and lane-group t (0..3), 16 bytes
 //   x[4t], x[4t+2], x[4t+1], x[4t+3], x[4t+16], x[4t+18], x[4t+17], x[4t+19]
-// Each thread moves groups of 8 consecutive values; the global loads of four
-// groups are issued together before any of them is stored.
+// Each thread moves groups of 8 consecutive values; the global loads of eight
+// groups (four for fp32) are issued together before any of them is stored.
 template <int XT>
 __device__ void load_x_window(uint8_t* xs, const void* x, int64_t K, int B, int c0, int nwin,
                               uint32_t term_stride, int tid) {
@@ -499,8 +535,8 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB) gemv_kernel(const Gemv
   }
 
   // -------------------------------------------------------------- consumers
-  const int cw = warp - 1;                // consumer index 0..7
-  const int ctid = threadIdx.x - 32;      // 0..255
+  const int cw = warp - 1;                // consumer index, also its share of a chunk
+  const int ctid = threadIdx.x - 32;      // 0 .. 32 * kConsumers - 1
   const int r = lane >> 2, t = lane & 3;  // fragment row group / thread in group
   const int bsel = min(r, a.B - 1);       // batch column this lane's B fragment reads
   bool ok = true;
@@ -561,8 +597,8 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB) gemv_kernel(const Gemv
       if constexpr (FMT == GQ_FMT_Q4_0) {
         const int nvalid = whole ? kSubPerWarp : tail_valid;
         if constexpr (ALIGNED) {
-          q40_chunk<XT, NB1, true>(acc, stg + r * kPitch, stg + (r + 8) * kPitch, xw, term_stride,
-                                   cw, t, nvalid);
+          q40_chunk<XT, NB1, true>(acc, stg + r * kPitch, stg + (r + 8) * kPitch, xw,
+                                   term_stride, cw, t, nvalid);
         } else {
           q40_chunk<XT, NB1, false>(acc, stg + r * kPitch + off0, stg + (r + 8) * kPitch + off1,
                                     xw, term_stride, cw, t, nvalid);
@@ -602,10 +638,9 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB) gemv_kernel(const Gemv
       }
       const int64_t ra = m0 + r, rbw = m0 + r + 8;
       if (NB1) {
-        if (t == 0) {
-          if (ra < a.M) store_elem(a.y, ra, s4[0], a.ytype);
-          if (rbw < a.M) store_elem(a.y, rbw, s4[2], a.ytype);
-        }
+        // lane t = 0 holds row r, lane t = 1 row r + 8 (scale_acc)
+        const int64_t row = (t == 0) ? ra : rbw;
+        if (t < 2 && row < a.M) store_elem(a.y, row, s4[0], a.ytype);
       } else {
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
@@ -627,8 +662,8 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB) gemv_kernel(const Gemv
 
 size_t gemv_smem_bytes(int B, int terms, int win) {
   return static_cast<size_t>(kStages) * kStageBytes +
-         static_cast<size_t>(terms) * win * B * kXStride +
-         2 * kConsumers * 32 * 4 * sizeof(float) + (2 * kStages + 1) * sizeof(uint64_t) + 16;
+         static_cast<size_t>(terms) * win * B * kXStride + kRedBytes +
+         (2 * kStages + 1) * sizeof(uint64_t) + 16;
 }
 
 template <int FMT, int XT, bool NB1, bool ALIGNED>
@@ -644,9 +679,9 @@ gq_status launch_gemv(GemvArgs a, cudaStream_t stream, bool pdl) {
   if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
   if (configured_dev != dev || smem > configured_smem) {
     // at least the common sizes, and always this launch's own requirement
-    const size_t want = smem > gemv_smem_bytes(1, kTerms, 1) + kXSmemMax
+    const size_t want = smem > gemv_smem_bytes(1, kTerms, 0) + kXSmemMax
                             ? smem
-                            : gemv_smem_bytes(1, kTerms, 1) + kXSmemMax;
+                            : gemv_smem_bytes(1, kTerms, 0) + kXSmemMax;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(want)) != cudaSuccess)
       return GQ_ERR_CUDA;
