@@ -23,12 +23,13 @@ GQ_F32, GQ_F16, GQ_BF16 = 0, 1, 2
 GQ_FMT_Q4_0, GQ_FMT_KSB = 0, 1
 GQ_DEV_NONFINITE, GQ_DEV_RANGE, GQ_DEV_TIMEOUT = 1, 2, 4
 GQ_GEMV_PDL = 1
+GQ_QUANT_REF_RULE = 1
 
 # every symbol include/gq.h declares
 EXPORTS = (
     "gq_abi_version", "gq_status_string", "gq_status_from_dev",
     "gq_q4_0_bytes", "gq_ksb_bytes",
-    "gq_quantize_q4_0", "gq_quantize_ksb",
+    "gq_quantize_q4_0", "gq_quantize_q4_0_ex", "gq_quantize_ksb",
     "gq_dequantize_q4_0", "gq_dequantize_ksb",
     "gq_gemv_workspace_bytes", "gq_gemv_q4_0", "gq_gemv_ksb",
     "gq_gemm_workspace_bytes", "gq_gemm_q4_0", "gq_gemm_ksb",
@@ -63,6 +64,8 @@ def _load() -> ctypes.CDLL:
         f = getattr(L, name)
         f.argtypes = [vp, i64, vp, vp, vp]
         f.restype = c_int
+    L.gq_quantize_q4_0_ex.argtypes = [vp, i64, vp, ctypes.c_uint, vp, vp]
+    L.gq_quantize_q4_0_ex.restype = c_int
     for name in ("gq_dequantize_q4_0", "gq_dequantize_ksb"):
         f = getattr(L, name)
         f.argtypes = [vp, i64, vp, vp]
@@ -145,6 +148,20 @@ def gq_quantize_q4_0(x: torch.Tensor, out: torch.Tensor | None = None,
                      dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """fp32 values (numel % 32 == 0) -> uint8 Q4_0 blocks (18 bytes per 32)."""
     return _quantize("gq_quantize_q4_0", gq_q4_0_bytes, x, out, dev_status, stream)
+
+
+def gq_quantize_q4_0_ex(x: torch.Tensor, flags: int, out: torch.Tensor | None = None,
+                        dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """gq_quantize_q4_0 with a rule flag (0, or GQ_QUANT_REF_RULE for the page's
+    reference quantizer: d = signed max / -8, codes min(15, trunc(x/d + 8.5)))."""
+    if x.dtype != torch.float32:
+        raise TypeError("quantizer input must be float32")
+    n = x.numel()
+    if out is None:
+        out = torch.empty(max(gq_q4_0_bytes(n), 0), dtype=torch.uint8, device=x.device)
+    _check(lib.gq_quantize_q4_0_ex(_ptr(x), n, _ptr(out), int(flags), _ptr(dev_status),
+                                   _stream(stream)), "gq_quantize_q4_0_ex")
+    return out
 
 
 def gq_quantize_ksb(x: torch.Tensor, out: torch.Tensor | None = None,

@@ -126,6 +126,62 @@ __device__ __forceinline__ void flush_tile(uint8_t* dst, const uint8_t* stage, i
   }
 }
 
+// ------------------------------------------- the page's reference Q4_0 rule
+// Q4_0 chapter 4.4 (its printed quantizer): the signed value of largest
+// magnitude (the first such value of the block on ties) sets d = max / -8;
+// with id = 1/d (0 when d is 0) code = min(15, trunc(x * id + 8.5)), the
+// product and the sum each rounded to fp32.  Dividing by -8 is exact, so d is
+// max * -0.125; a NaN value never becomes the max.
+
+// 64-bit ordering key of value v at block position i: larger magnitude first,
+// then the earlier position, the sign in bit 0; 0 for NaN and for zeros, so
+// that a block of zeros takes max = +0 as the page's loop (which starts from
+// 0 and only replaces it on a strictly larger magnitude) does.
+__device__ __forceinline__ unsigned long long smax_key(float v, int i) {
+  const uint32_t bits = __float_as_uint(v), mag = bits & 0x7FFFFFFFu;
+  if (isnan(v) || mag == 0u) return 0ull;
+  return (static_cast<unsigned long long>(mag) << 32) | (static_cast<uint32_t>(31 - i) << 1) |
+         (bits >> 31);
+}
+__device__ __forceinline__ float key_value(unsigned long long k) {
+  const uint32_t mag = static_cast<uint32_t>(k >> 32), sign = static_cast<uint32_t>(k) & 1u;
+  return __uint_as_float(mag | (sign << 31));
+}
+
+// The four qs bytes of one lane (weights 4t..4t+3 in lo, 16+4t.. in hi)
+// under the reference rule, with id = 1/d.
+__device__ __forceinline__ uint32_t ref_code(float v, float id) {
+  const float tt = __fadd_rn(__fmul_rn(v, id), 8.5f);
+  const int c = (tt >= 0.0f && tt < 1e9f) ? __float2int_rz(tt) : 0;
+  return static_cast<uint32_t>(c < 15 ? c : 15);
+}
+__device__ __forceinline__ uint32_t ref_qs_bytes(float4 lo, float4 hi, float id) {
+  return (ref_code(lo.x, id) | (ref_code(hi.x, id) << 4)) |
+         ((ref_code(lo.y, id) | (ref_code(hi.y, id) << 4)) << 8) |
+         ((ref_code(lo.z, id) | (ref_code(hi.z, id) << 4)) << 16) |
+         ((ref_code(lo.w, id) | (ref_code(hi.w, id) << 4)) << 24);
+}
+
+// Scale of the reference rule for the block whose values this lane group of
+// four holds (lane t: positions 4t..4t+3 and 16+4t..19+4t).
+__device__ __forceinline__ float ref_scale(float4 lo, float4 hi, int t) {
+  unsigned long long k = smax_key(lo.x, 4 * t);
+  const float lv[4] = {lo.x, lo.y, lo.z, lo.w}, hv[4] = {hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const unsigned long long a = smax_key(lv[i], 4 * t + i);
+    const unsigned long long b = smax_key(hv[i], 16 + 4 * t + i);
+    k = a > k ? a : k;
+    k = b > k ? b : k;
+  }
+#pragma unroll
+  for (int o = 1; o <= 2; o <<= 1) {
+    const unsigned long long other = __shfl_xor_sync(0xFFFFFFFFu, k, o);
+    k = other > k ? other : k;
+  }
+  return __fmul_rn(key_value(k), -0.125f);
+}
+
 // ---------------------------------------------------------------- Q4_0 quantize
 // CTA tile: 128 blocks (4096 floats).  Four lanes share a block: lane t of a
 // block holds weights 4t..4t+3 and 16+4t..19+4t, the two halves whose codes
@@ -135,6 +191,7 @@ __device__ __forceinline__ void flush_tile(uint8_t* dst, const uint8_t* stage, i
 // keeps 64 B of reads in flight while it computes.
 constexpr int kQ0Tile = 128;
 
+template <bool REF_RULE>
 __global__ void __launch_bounds__(kQThreads)
     quantize_q4_0_kernel(const float* __restrict__ x, int64_t nblk, uint8_t* __restrict__ out,
                          int* dev_status) {
@@ -167,10 +224,17 @@ __global__ void __launch_bounds__(kQThreads)
       const int bl = warp * 16 + h * 8 + (lane >> 2);
       const float own = absmax8(lo[h], hi[h]);
       if (!(own < INFINITY)) flags |= GQ_DEV_NONFINITE;
-      const __half dh = scale_over(group4_max(own), 7.0f, kInv7);
-      const float d = __half2float(dh);
+      __half dh;
+      uint32_t b;
+      if constexpr (REF_RULE) {
+        const float d = ref_scale(lo[h], hi[h], t);
+        dh = __float2half_rn(d);
+        b = ref_qs_bytes(lo[h], hi[h], d != 0.0f ? __frcp_rn(d) : 0.0f);
+      } else {
+        dh = scale_over(group4_max(own), 7.0f, kInv7);
+        b = qs_bytes(lo[h], hi[h], __half2float(dh));
+      }
       if (__hisinf(dh)) flags |= GQ_DEV_RANGE;
-      const uint32_t b = qs_bytes(lo[h], hi[h], d);
       if (bl < nb) {
         uint8_t* blk = stage + bl * 18;
         if (t == 0) st_u16(blk, __half_as_ushort(dh));
@@ -377,14 +441,27 @@ using namespace gq;
 
 extern "C" {
 
-GQ_API gq_status gq_quantize_q4_0(const float* x, int64_t n, void* out, int* dev_status,
-                                  void* stream) {
+GQ_API gq_status gq_quantize_q4_0_ex(const float* x, int64_t n, void* out, unsigned flags,
+                                     int* dev_status, void* stream) {
+  if (flags & ~GQ_QUANT_REF_RULE) return GQ_ERR_INVALID_ARG;
   gq_status s = check_common(x, n, 32, out, dev_status);
   if (s != GQ_OK || n == 0) return s;
   const int64_t nblk = n / 32;
-  const dim3 grid(resident_grid(quantize_q4_0_kernel, (nblk + kQ0Tile - 1) / kQ0Tile));
-  return launch(quantize_q4_0_kernel, grid, dim3(kQThreads), 0, as_stream(stream), false, x, nblk,
-                static_cast<uint8_t*>(out), dev_status);
+  const int64_t tiles = (nblk + kQ0Tile - 1) / kQ0Tile;
+  uint8_t* o = static_cast<uint8_t*>(out);
+  if (flags & GQ_QUANT_REF_RULE) {
+    const dim3 grid(resident_grid(quantize_q4_0_kernel<true>, tiles));
+    return launch(quantize_q4_0_kernel<true>, grid, dim3(kQThreads), 0, as_stream(stream), false,
+                  x, nblk, o, dev_status);
+  }
+  const dim3 grid(resident_grid(quantize_q4_0_kernel<false>, tiles));
+  return launch(quantize_q4_0_kernel<false>, grid, dim3(kQThreads), 0, as_stream(stream), false, x,
+                nblk, o, dev_status);
+}
+
+GQ_API gq_status gq_quantize_q4_0(const float* x, int64_t n, void* out, int* dev_status,
+                                  void* stream) {
+  return gq_quantize_q4_0_ex(x, n, out, 0u, dev_status, stream);
 }
 
 GQ_API gq_status gq_quantize_ksb(const float* x, int64_t n, void* out, int* dev_status,

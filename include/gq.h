@@ -118,6 +118,19 @@ GQ_API size_t gq_ksb_bytes(int64_t n);
 GQ_API gq_status gq_quantize_q4_0(const float* x, int64_t n, void* out,
                                   int* dev_status, void* stream);
 
+/* gq_quantize_q4_0 with a choice of rule.  flags: 0 (the rule above, the same
+ * as gq_quantize_q4_0) or GQ_QUANT_REF_RULE, the page's own reference
+ * quantizer (Q4_0 chapter 4.4, the printed quantizer, and its outlier demo in
+ * 4.5): the signed value of largest magnitude (the first on ties; +0 for a
+ * block of zeros) sets d = max / -8, and with id = 1/d (0 when d is 0) each
+ * code is min(15, trunc(x * id + 8.5)), the product and the sum each rounded
+ * to fp32.  The stored scale is FP16(d).  Other flag bits give
+ * GQ_ERR_INVALID_ARG.  Arguments and status as for gq_quantize_q4_0
+ * (GQ_DEV_RANGE when FP16(d) is infinite). */
+#define GQ_QUANT_REF_RULE 1u
+GQ_API gq_status gq_quantize_q4_0_ex(const float* x, int64_t n, void* out, unsigned flags,
+                                     int* dev_status, void* stream);
+
 /* Quantize n fp32 values into KSB super-blocks (K-quants post, "套娃": the
  * eight sub-block scales are quantized to INT8 against an FP16 super-scale).
  *   n % 256 == 0; out holds gq_ksb_bytes(n) bytes.  dev_status as above. */

@@ -67,6 +67,18 @@ def test_quantize_validation(name, block):
     assert f(A, block, A, A + 1, None) == ALIGN          # dev_status must be int-aligned
 
 
+def test_quantize_rule_flag_validation():
+    f = gq.lib.gq_quantize_q4_0_ex
+    for flags in (2, 4, 0x80000000, 0xFFFFFFFF):
+        assert f(A, 32, A, flags, None, None) == INVALID   # unknown rule bits first
+    for flags in (0, gq.GQ_QUANT_REF_RULE):
+        assert f(A, -32, A, flags, None, None) == INVALID
+        assert f(A, 33, A, flags, None, None) == SHAPE
+        assert f(None, 0, None, flags, None, None) == GQ_OK
+        assert f(A + 4, 32, A, flags, None, None) == ALIGN
+        assert f(A, 32, A, flags, A + 1, None) == ALIGN
+
+
 @pytest.mark.parametrize("name,block", [("gq_dequantize_q4_0", 32), ("gq_dequantize_ksb", 256)])
 def test_dequantize_validation(name, block):
     f = getattr(gq.lib, name)

@@ -268,3 +268,90 @@ def test_ksb_subscales_at_half_integers():
     got, st = gpu_quantize(KSB, torch.from_numpy(x))
     assert st == flags == 0
     assert_bytes_equal(got, want, 138)
+
+
+# ------------------------------------------------------------------------
+# The page's reference quantizer (Q4_0 chapter 4.4; GQ_QUANT_REF_RULE)
+
+def gpu_quantize_ref(x: np.ndarray):
+    xt = torch.from_numpy(np.ascontiguousarray(x, np.float32).ravel()).cuda()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q = gq.gq_quantize_q4_0_ex(xt, gq.GQ_QUANT_REF_RULE, dev_status=st)
+    torch.cuda.synchronize()
+    return q.cpu().numpy(), int(st.item())
+
+
+@pytest.mark.parametrize("rows,cols,seed", [(64, 1024, 0), (4096, 4096, 1), (7, 96, 2)])
+def test_ref_rule_random(rows, cols, seed):
+    w = synth.gaussian_weights(rows, cols, seed=seed).numpy()
+    want, flags = oracle.quantize_q4_0(w.ravel(), rule=oracle.RULE_LLAMA)
+    got, st = gpu_quantize_ref(w)
+    assert st == flags
+    assert_bytes_equal(got, want, 18)
+
+
+def test_ref_rule_outlier_demo_and_ties():
+    rng = np.random.default_rng(5)
+    blocks = []
+    # the page's outlier demo (section 4.5): 31 small values and one 10
+    blocks.append(np.array([0.01 * (i - 15) / 15 for i in range(31)] + [10.0], np.float32))
+    # equal magnitudes of both signs: the first one sets the sign of d
+    for _ in range(200):
+        b = rng.uniform(-1, 1, 32).astype(np.float32)
+        m = np.float32(rng.uniform(1, 4))
+        i, j = sorted(rng.choice(32, 2, replace=False))
+        b[i], b[j] = (m, -m) if rng.random() < 0.5 else (-m, m)
+        blocks.append(b)
+    # zeros (signed and unsigned), a single value, subnormals, huge values
+    blocks.append(np.zeros(32, np.float32))
+    blocks.append(-np.zeros(32, np.float32))
+    z = np.zeros(32, np.float32); z[17] = -3.0; blocks.append(z)
+    blocks.append((rng.standard_normal(32) * 1e-40).astype(np.float32))
+    blocks.append((rng.standard_normal(32) * 1e30).astype(np.float32))
+    x = np.stack(blocks)
+    want, flags = oracle.quantize_q4_0(x.ravel(), rule=oracle.RULE_LLAMA)
+    got, st = gpu_quantize_ref(x)
+    assert st == flags
+    assert_bytes_equal(got, want, 18)
+
+
+def test_ref_rule_code_boundaries():
+    # values placed so that x * id + 8.5 lands on and beside integers, where
+    # truncation decides the code
+    rng = np.random.default_rng(11)
+    nb = 20000
+    vmax = (2.0 ** rng.uniform(-20, 10, nb)).astype(np.float32) * np.where(
+        rng.random(nb) < 0.5, 1, -1).astype(np.float32)
+    d = vmax / np.float32(-8.0)
+    x = np.empty((nb, 32), np.float32)
+    for b in range(nb):
+        k = rng.integers(-8, 8, 32).astype(np.float64)
+        v = ((k - 0.5) * np.float64(d[b])).astype(np.float32)     # x * id + 8.5 ~ k + 8
+        nudge = rng.integers(-2, 3, 32)
+        for i in range(32):
+            for _ in range(abs(int(nudge[i]))):
+                v[i] = np.nextafter(v[i], np.float32(np.inf if nudge[i] > 0 else -np.inf))
+        v = np.where(np.abs(v) < np.abs(vmax[b]), v, np.float32(0.0))
+        v[rng.integers(0, 32)] = vmax[b]
+        x[b] = v
+    want, flags = oracle.quantize_q4_0(x.ravel(), rule=oracle.RULE_LLAMA)
+    got, st = gpu_quantize_ref(x)
+    assert st == flags
+    assert_bytes_equal(got, want, 18)
+
+
+def test_ref_rule_flags_and_default_unchanged():
+    x = np.zeros(32 * 64, np.float32)
+    x[40] = 8 * 70000.0                      # |d| = 70000 overflows FP16
+    _, st = gpu_quantize_ref(x)
+    _, flags = oracle.quantize_q4_0(x, rule=oracle.RULE_LLAMA)
+    assert st == flags == gq.GQ_DEV_RANGE
+    x[40] = 1.0
+    x[300] = np.nan
+    _, st = gpu_quantize_ref(x)
+    assert st & gq.GQ_DEV_NONFINITE
+    # flags = 0 is the default rule, byte for byte
+    w = synth.gaussian_weights(32, 512, seed=3)
+    a = gq.gq_quantize_q4_0_ex(w.view(-1).cuda(), 0).cpu().numpy()
+    b = gq.gq_quantize_q4_0(w.view(-1).cuda()).cpu().numpy()
+    assert np.array_equal(a, b)
