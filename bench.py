@@ -515,6 +515,19 @@ def run_suite(path):
               "ms": round(ms, 3), "weight_gbs": round(total / (ms * 1e-3) / 1e9, 1),
               "frac_of_peak": round(total / (ms * 1e-3) / 1e9 / peak, 4),
               "matrices_per_s": round(224 / (ms * 1e-3), 1)})
+        # the same 224 products as one grouped call (one launch, x loaded once per CTA)
+        fg = gq.gq_gemv_q4_0_grouped if fmt == "q4_0" else gq.gq_gemv_ksb_grouped
+        outs = [torch.empty((1, M), dtype=torch.float16, device=dev) for _, M, _ in mats]
+        Ws, Ms = [m[0] for m in mats], [m[1] for m in mats]
+        ms = _graph_ms_per_launch(
+            lambda: fg(Ws, Ms, 4096, x, outs=outs, flags=gq.GQ_GEMV_PDL), 1, 5)
+        emit({"row": "model_stream_grouped", "workload": "32 layers x (4 x 4096x4096 + 3 x "
+              "11008x4096), 224 batch-1 GEMVs in one grouped call", "format": fmt,
+              "weight_bytes": total, "ms": round(ms, 3),
+              "weight_gbs": round(total / (ms * 1e-3) / 1e9, 1),
+              "frac_of_peak": round(total / (ms * 1e-3) / 1e9 / peak, 4),
+              "matrices_per_s": round(224 / (ms * 1e-3), 1)})
+        del Ws, outs
         del mats
         torch.cuda.empty_cache()
 

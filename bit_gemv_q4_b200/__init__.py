@@ -32,6 +32,7 @@ EXPORTS = (
     "gq_quantize_q4_0", "gq_quantize_q4_0_ex", "gq_quantize_ksb",
     "gq_dequantize_q4_0", "gq_dequantize_ksb",
     "gq_gemv_workspace_bytes", "gq_gemv_q4_0", "gq_gemv_ksb",
+    "gq_gemv_q4_0_grouped", "gq_gemv_ksb_grouped",
     "gq_gemm_workspace_bytes", "gq_gemm_q4_0", "gq_gemm_ksb",
     "gq_selftest_gemv_timeout", "gq_gemv_q4_0_noalloc",
 )
@@ -76,6 +77,10 @@ def _load() -> ctypes.CDLL:
         f = getattr(L, name)
         f.argtypes = [vp, i64, i64, vp, c_int, i64, vp, c_int, vp, ctypes.c_size_t, c_uint, vp,
                       vp]
+        f.restype = c_int
+    for name in ("gq_gemv_q4_0_grouped", "gq_gemv_ksb_grouped"):
+        f = getattr(L, name)
+        f.argtypes = [vp, c_int, i64, vp, c_int, i64, c_int, c_uint, vp, vp]
         f.restype = c_int
     L.gq_gemm_workspace_bytes.argtypes = [c_int, i64, i64, i64]
     L.gq_gemm_workspace_bytes.restype = ctypes.c_size_t
@@ -249,6 +254,48 @@ def gq_gemv_ksb(W: torch.Tensor, M: int, K: int, x: torch.Tensor, y_dtype=torch.
     """y[B, M] = W_hat[M, K] @ x[B, K]^T for super-block weights; B in 1..8."""
     return _gemv("gq_gemv_ksb", GQ_FMT_KSB, W, M, K, x, y_dtype, out, workspace, flags,
                  dev_status, stream)
+
+
+class GemvDesc(ctypes.Structure):
+    """gq_gemv_desc: one matrix of a grouped GEMV."""
+    _fields_ = [("W", ctypes.c_void_p), ("M", ctypes.c_int64), ("y", ctypes.c_void_p)]
+
+
+def _gemv_grouped(name: str, Ws, Ms, K: int, x: torch.Tensor, y_dtype, outs, flags: int,
+                  dev_status, stream):
+    if len(Ws) != len(Ms):
+        raise ValueError("one M per matrix")
+    x2 = x if x.dim() == 2 else x.reshape(1, -1)
+    B = x2.shape[0]
+    if x2.shape[1] != K:
+        raise ValueError(f"x has {x2.shape[1]} columns, expected K={K}")
+    if x2.dtype not in _DTYPE_CODE or y_dtype not in _DTYPE_CODE:
+        raise TypeError("activations and outputs must be float32, float16 or bfloat16")
+    if outs is None:
+        outs = [torch.empty((B, int(M)), dtype=y_dtype, device=x2.device) for M in Ms]
+    if len(outs) != len(Ws) or any(o.dtype != outs[0].dtype for o in outs):
+        raise ValueError("one output per matrix, all of one dtype")
+    descs = (GemvDesc * len(Ws))(*[GemvDesc(_ptr(W), int(M), _ptr(o))
+                                   for W, M, o in zip(Ws, Ms, outs)])
+    ytype = _DTYPE_CODE[outs[0].dtype] if outs else _DTYPE_CODE[y_dtype]
+    _check(getattr(lib, name)(ctypes.cast(descs, ctypes.c_void_p), len(Ws), int(K), _ptr(x2),
+                              _DTYPE_CODE[x2.dtype], B, ytype,
+                              int(flags), _ptr(dev_status), _stream(stream)), name)
+    return outs
+
+
+def gq_gemv_q4_0_grouped(Ws, Ms, K: int, x: torch.Tensor, y_dtype=torch.float16, outs=None,
+                         flags: int = 0, dev_status: torch.Tensor | None = None, stream=None):
+    """[y_i = W_hat_i @ x^T for each Q4_0 matrix W_i (M_i x K)], one shared x [B, K]."""
+    return _gemv_grouped("gq_gemv_q4_0_grouped", Ws, Ms, K, x, y_dtype, outs, flags,
+                         dev_status, stream)
+
+
+def gq_gemv_ksb_grouped(Ws, Ms, K: int, x: torch.Tensor, y_dtype=torch.float16, outs=None,
+                        flags: int = 0, dev_status: torch.Tensor | None = None, stream=None):
+    """[y_i = W_hat_i @ x^T for each super-block matrix W_i (M_i x K)], one shared x."""
+    return _gemv_grouped("gq_gemv_ksb_grouped", Ws, Ms, K, x, y_dtype, outs, flags,
+                         dev_status, stream)
 
 
 def gq_gemm_workspace_bytes(fmt: int, M: int, K: int, B: int) -> int:

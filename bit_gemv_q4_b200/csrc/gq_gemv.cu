@@ -106,6 +106,45 @@ struct GemvArgs {
   int skip_first;  // self-test only: never fill the first stage, so waits run out
 };
 
+// Matrices of one launch.  A single product reads W, M and y from GemvArgs
+// (NoTable); a grouped product (several matrices sharing K and x) numbers
+// the 16-row groups of all its matrices consecutively and finds a group's
+// matrix in a table passed by value (GemvTable, read from the kernel's
+// parameter space).
+struct NoTable {
+  int unused;
+};
+constexpr int kMaxMats = 256;  // matrices per grouped launch
+struct GemvMat {
+  const uint8_t* W;
+  void* y;
+  int64_t M;
+  int gend;  // groups of matrices 0..i
+  int pad;
+};
+struct GemvTable {
+  GemvMat m[kMaxMats];
+};
+
+struct Unit {
+  const uint8_t* W;
+  void* y;
+  int64_t M, m0;  // the matrix and the first row of the group
+};
+
+// The matrix of group g.  Each CTA visits groups in increasing order, so
+// its cursor mi only moves forward.
+template <class Tbl>
+__device__ __forceinline__ Unit unit_of(const GemvArgs& a, const Tbl& tbl, int g, int& mi) {
+  if constexpr (sizeof(Tbl) == sizeof(NoTable)) {
+    return Unit{a.W, a.y, a.M, static_cast<int64_t>(g) * kRows};
+  } else {
+    while (g >= tbl.m[mi].gend) ++mi;
+    const int gb = mi ? tbl.m[mi - 1].gend : 0;
+    return Unit{tbl.m[mi].W, tbl.m[mi].y, tbl.m[mi].M, static_cast<int64_t>(g - gb) * kRows};
+  }
+}
+
 // ---- decode 8 codes (one 32-bit word = qs[4t..4t+3]) into four A registers
 // holding (code - 8) as packed halves:
 //   r0 = (w[4t],    w[4t+2])     r1 = (w[4t+16], w[4t+18])
@@ -437,8 +476,9 @@ __device__ void load_x_window(uint8_t* xs, const void* x, int64_t K, int B, int 
   }
 }
 
-template <int FMT, int XT, bool NB1, bool ALIGNED>
-__global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB) gemv_kernel(const GemvArgs a) {
+template <int FMT, int XT, bool NB1, bool ALIGNED, class Tbl>
+__global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
+    gemv_kernel(const GemvArgs a, const __grid_constant__ Tbl tbl) {
   constexpr int kBlkW = Fmt<FMT>::kBlkW, kBlkB = Fmt<FMT>::kBlkB;
   constexpr int kTerms = (XT == XT_F32) ? 3 : 1;
   constexpr int kBlkPerChunk = kChunkW / kBlkW;
@@ -477,10 +517,12 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB) gemv_kernel(const Gemv
     uint32_t ph = 0;     // its phase parity
     bool ok = true;
     const uint32_t tail_bytes = static_cast<uint32_t>((nblk_row - nfull * kBlkPerChunk) * kBlkB);
+    int pmi = 0;  // matrix cursor
     for (int g = blockIdx.x; g < a.ngroups && ok; g += gridDim.x) {
-      const int64_t m0 = static_cast<int64_t>(g) * kRows;
-      const bool row_ok = lane < kRows && m0 + lane < a.M;
-      uintptr_t src = reinterpret_cast<uintptr_t>(a.W) +
+      const Unit un = unit_of(a, tbl, g, pmi);
+      const int64_t m0 = un.m0;
+      const bool row_ok = lane < kRows && m0 + lane < un.M;
+      uintptr_t src = reinterpret_cast<uintptr_t>(un.W) +
                       static_cast<uintptr_t>((m0 + (row_ok ? lane : 0)) * a.rowbytes);
       for (int c = 0; c < a.nchunks; ++c, ++issued, src += kChunkBytes) {
         if (!mbar_wait(&empty[s], ph ^ 1u, a.budget) ||
@@ -571,14 +613,17 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB) gemv_kernel(const Gemv
   int s = 0;        // stage of the next use
   uint32_t ph = 0;  // its phase parity
   int gi = 0;       // groups done by this CTA
+  int cmi = 0;  // matrix cursor
   for (int g = blockIdx.x; g < a.ngroups && ok; g += gridDim.x, ++gi) {
-    const int64_t m0 = static_cast<int64_t>(g) * kRows;
+    const Unit un = unit_of(a, tbl, g, cmi);
+    const int64_t m0 = un.m0;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     // offset of row r's (and r+8's) first byte inside its 16-byte granule
     uint32_t off0 = static_cast<uint32_t>(
-        (reinterpret_cast<uintptr_t>(a.W) + static_cast<uintptr_t>((m0 + r) * a.rowbytes)) & 15u);
+        (reinterpret_cast<uintptr_t>(un.W) + static_cast<uintptr_t>((m0 + r) * a.rowbytes)) & 15u);
     uint32_t off1 = static_cast<uint32_t>(
-        (reinterpret_cast<uintptr_t>(a.W) + static_cast<uintptr_t>((m0 + r + 8) * a.rowbytes)) & 15u);
+        (reinterpret_cast<uintptr_t>(un.W) + static_cast<uintptr_t>((m0 + r + 8) * a.rowbytes)) &
+        15u);
     uint32_t xw = x_lane;
     int cw_in_win = 0;
     for (int c = 0; c < a.nchunks; ++c) {
@@ -640,14 +685,14 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB) gemv_kernel(const Gemv
       if (NB1) {
         // lane t = 0 holds row r, lane t = 1 row r + 8 (scale_acc)
         const int64_t row = (t == 0) ? ra : rbw;
-        if (t < 2 && row < a.M) store_elem(a.y, row, s4[0], a.ytype);
+        if (t < 2 && row < un.M) store_elem(un.y, row, s4[0], a.ytype);
       } else {
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           const int col = 2 * t + i;
           if (col < a.B) {
-            if (ra < a.M) store_elem(a.y, col * a.M + ra, s4[i], a.ytype);
-            if (rbw < a.M) store_elem(a.y, col * a.M + rbw, s4[2 + i], a.ytype);
+            if (ra < un.M) store_elem(un.y, col * un.M + ra, s4[i], a.ytype);
+            if (rbw < un.M) store_elem(un.y, col * un.M + rbw, s4[2 + i], a.ytype);
           }
         }
       }
@@ -666,10 +711,10 @@ size_t gemv_smem_bytes(int B, int terms, int win) {
          (2 * kStages + 1) * sizeof(uint64_t) + 16;
 }
 
-template <int FMT, int XT, bool NB1, bool ALIGNED>
-gq_status launch_gemv(GemvArgs a, cudaStream_t stream, bool pdl) {
+template <int FMT, int XT, bool NB1, bool ALIGNED, class Tbl>
+gq_status launch_gemv(const GemvArgs& a, const Tbl& tbl, cudaStream_t stream, bool pdl) {
   constexpr int kTerms = (XT == XT_F32) ? 3 : 1;
-  auto kern = gemv_kernel<FMT, XT, NB1, ALIGNED>;
+  auto kern = gemv_kernel<FMT, XT, NB1, ALIGNED, Tbl>;
   const size_t smem = gemv_smem_bytes(a.B, kTerms, a.win);
   static int configured_dev = -1;
   static size_t configured_smem = 0;
@@ -699,20 +744,52 @@ gq_status launch_gemv(GemvArgs a, cudaStream_t stream, bool pdl) {
   }
   const int64_t slots = static_cast<int64_t>(sm_count()) * occupancy;
   const int grid = static_cast<int>(a.ngroups < slots ? a.ngroups : slots);
-  return launch(kern, dim3(grid), dim3(kThreads), smem, stream, pdl, a);
+  return launch(kern, dim3(grid), dim3(kThreads), smem, stream, pdl, a, tbl);
 }
 
-template <int FMT, int XT>
-gq_status dispatch_gemv(const GemvArgs& a, cudaStream_t s, bool pdl) {
+// w_aligned: every matrix of the launch starts on a 16-byte boundary.
+template <int FMT, int XT, class Tbl>
+gq_status dispatch_gemv(const GemvArgs& a, const Tbl& tbl, bool w_aligned, cudaStream_t s,
+                        bool pdl) {
   const bool nb1 = (a.B == 1);
-  const bool aligned = (FMT == GQ_FMT_Q4_0) && (a.rowbytes % 16 == 0) &&
-                       (reinterpret_cast<uintptr_t>(a.W) % 16 == 0);
+  const bool aligned = (FMT == GQ_FMT_Q4_0) && (a.rowbytes % 16 == 0) && w_aligned;
   if (nb1) {
-    return aligned ? launch_gemv<FMT, XT, true, true>(a, s, pdl)
-                   : launch_gemv<FMT, XT, true, false>(a, s, pdl);
+    return aligned ? launch_gemv<FMT, XT, true, true>(a, tbl, s, pdl)
+                   : launch_gemv<FMT, XT, true, false>(a, tbl, s, pdl);
   }
-  return aligned ? launch_gemv<FMT, XT, false, true>(a, s, pdl)
-                 : launch_gemv<FMT, XT, false, false>(a, s, pdl);
+  return aligned ? launch_gemv<FMT, XT, false, true>(a, tbl, s, pdl)
+                 : launch_gemv<FMT, XT, false, false>(a, tbl, s, pdl);
+}
+
+template <int FMT, class Tbl>
+gq_status dispatch_xt(const GemvArgs& a, const Tbl& tbl, int xt, bool w_aligned, cudaStream_t s,
+                      bool pdl) {
+  switch (xt) {
+    case GQ_F16: return dispatch_gemv<FMT, XT_F16>(a, tbl, w_aligned, s, pdl);
+    case GQ_BF16: return dispatch_gemv<FMT, XT_BF16>(a, tbl, w_aligned, s, pdl);
+    default: return dispatch_gemv<FMT, XT_F32>(a, tbl, w_aligned, s, pdl);
+  }
+}
+
+// The fields of GemvArgs that depend only on K, B and the dtypes.
+template <int FMT>
+void fill_common(GemvArgs& a, int64_t K, const void* x, int xt, int64_t B, int yt,
+                 int* dev_status, long long budget) {
+  constexpr int kBlkW = Fmt<FMT>::kBlkW, kBlkB = Fmt<FMT>::kBlkB;
+  a.K = K;
+  a.rowbytes = K / kBlkW * kBlkB;
+  a.x = x;
+  a.dev_status = dev_status;
+  a.budget = budget;
+  a.B = static_cast<int>(B);
+  a.ytype = yt;
+  a.nchunks = static_cast<int>((K + kChunkW - 1) / kChunkW);
+  a.skip_first = 0;
+  const int terms = (xt == GQ_F32) ? 3 : 1;
+  int win = kXSmemMax / (terms * a.B * kXStride);
+  if (win < 1) win = 1;
+  if (win > a.nchunks) win = a.nchunks;
+  a.win = win;
 }
 
 template <int FMT>
@@ -720,7 +797,7 @@ gq_status gemv_entry(const void* W, int64_t M, int64_t K, const void* x, int xt,
                      void* y, int yt, void* workspace, size_t ws_bytes, unsigned flags,
                      int* dev_status, void* stream, long long budget = kWaitBudget,
                      int skip_first = 0) {
-  constexpr int kBlkW = Fmt<FMT>::kBlkW, kBlkB = Fmt<FMT>::kBlkB;
+  constexpr int kBlkW = Fmt<FMT>::kBlkW;
   if (M < 0 || K < 0 || B < 0) return GQ_ERR_INVALID_ARG;
   if (!valid_act_dtype(xt) || !valid_act_dtype(yt)) return GQ_ERR_DTYPE;
   if (flags & ~GQ_GEMV_PDL) return GQ_ERR_INVALID_ARG;
@@ -740,34 +817,82 @@ gq_status gemv_entry(const void* W, int64_t M, int64_t K, const void* x, int xt,
   if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return GQ_ERR_ALIGNMENT;
 
   GemvArgs a;
+  fill_common<FMT>(a, K, x, xt, B, yt, dev_status, budget);
   a.W = static_cast<const uint8_t*>(W);
   a.M = M;
-  a.K = K;
-  a.rowbytes = K / kBlkW * kBlkB;
-  a.x = x;
   a.y = y;
-  a.dev_status = dev_status;
-  a.budget = budget;
-  a.B = static_cast<int>(B);
-  a.ytype = yt;
-  a.nchunks = static_cast<int>((K + kChunkW - 1) / kChunkW);
   a.ngroups = static_cast<int>((M + kRows - 1) / kRows);
   a.skip_first = skip_first;
-  const int terms = (xt == GQ_F32) ? 3 : 1;
-  int win = kXSmemMax / (terms * a.B * kXStride);
-  if (win < 1) win = 1;
-  if (win > a.nchunks) win = a.nchunks;
-  a.win = win;
 
   const bool pdl = (flags & GQ_GEMV_PDL) != 0;
   cudaStream_t s = as_stream(stream);
   if (workspace && ws_bytes && !skip_first && i8_eligible(FMT, M, K, B, xt, W))
     return i8_gemv(W, M, K, x, y, yt, workspace, ws_bytes, pdl, dev_status, s);
-  switch (xt) {
-    case GQ_F16: return dispatch_gemv<FMT, XT_F16>(a, s, pdl);
-    case GQ_BF16: return dispatch_gemv<FMT, XT_BF16>(a, s, pdl);
-    default: return dispatch_gemv<FMT, XT_F32>(a, s, pdl);
+  return dispatch_xt<FMT>(a, NoTable{0}, xt, !misaligned16(W), s, pdl);
+}
+
+// Several matrices that share K and the activations x: y_i = W_i x for each
+// descriptor, in launches of up to kMaxMats matrices whose CTAs stream the
+// groups of all their matrices back to back.
+template <int FMT>
+gq_status gemv_grouped_entry(const gq_gemv_desc* mats, int count, int64_t K, const void* x,
+                             int xt, int64_t B, int yt, unsigned flags, int* dev_status,
+                             void* stream) {
+  constexpr int kBlkW = Fmt<FMT>::kBlkW;
+  if (count < 0 || K < 0 || B < 0) return GQ_ERR_INVALID_ARG;
+  if (count > 0 && !mats) return GQ_ERR_INVALID_ARG;
+  if (!valid_act_dtype(xt) || !valid_act_dtype(yt)) return GQ_ERR_DTYPE;
+  if (flags & ~GQ_GEMV_PDL) return GQ_ERR_INVALID_ARG;
+  if (K % kBlkW) return GQ_ERR_SHAPE;
+  if (B > 8 || K > (1LL << 24)) return GQ_ERR_SHAPE;
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return GQ_ERR_ALIGNMENT;
+  int64_t groups = 0;
+  for (int i = 0; i < count; ++i) {
+    const gq_gemv_desc& d = mats[i];
+    if (d.M < 0) return GQ_ERR_INVALID_ARG;
+    if (d.M > 0x7FFFFFFFLL) return GQ_ERR_SHAPE;
+    if (d.M == 0) continue;
+    if (!d.y || (K > 0 && !d.W)) return GQ_ERR_INVALID_ARG;
+    if (misaligned16(d.y) || misaligned16(d.W)) return GQ_ERR_ALIGNMENT;
+    groups += (d.M + kRows - 1) / kRows;
   }
+  if (groups > 0x7FFFFFFFLL) return GQ_ERR_SHAPE;
+  if (B == 0 || groups == 0) return GQ_OK;
+  cudaStream_t s = as_stream(stream);
+  if (K == 0) {
+    for (int i = 0; i < count; ++i)
+      if (mats[i].M > 0 && cudaMemsetAsync(mats[i].y, 0,
+                                           static_cast<size_t>(B * mats[i].M * dtype_size(yt)),
+                                           s) != cudaSuccess)
+        return GQ_ERR_CUDA;
+    return GQ_OK;
+  }
+  if (!x) return GQ_ERR_INVALID_ARG;
+  if (misaligned16(x)) return GQ_ERR_ALIGNMENT;
+
+  GemvArgs a;
+  fill_common<FMT>(a, K, x, xt, B, yt, dev_status, kWaitBudget);
+  a.W = nullptr;
+  a.M = 0;
+  a.y = nullptr;
+  const bool pdl = (flags & GQ_GEMV_PDL) != 0;
+  GemvTable tbl{};  // one launch's table, passed to the kernel by value
+  int i = 0;
+  while (i < count) {
+    int n = 0, g = 0;
+    for (; i < count && n < kMaxMats; ++i) {
+      const gq_gemv_desc& d = mats[i];
+      if (d.M == 0) continue;
+      g += static_cast<int>((d.M + kRows - 1) / kRows);
+      tbl.m[n] = GemvMat{static_cast<const uint8_t*>(d.W), d.y, d.M, g, 0};
+      ++n;
+    }
+    if (n == 0) break;
+    a.ngroups = g;
+    const gq_status st = dispatch_xt<FMT>(a, tbl, xt, true, s, pdl);
+    if (st != GQ_OK) return st;
+  }
+  return GQ_OK;
 }
 
 }  // namespace
@@ -795,6 +920,20 @@ GQ_API gq_status gq_gemv_ksb(const void* W, int64_t M, int64_t K, const void* x,
                              unsigned flags, int* dev_status, void* stream) {
   return gq::gemv_entry<GQ_FMT_KSB>(W, M, K, x, x_dtype, B, y, y_dtype, workspace, ws_bytes,
                                     flags, dev_status, stream);
+}
+
+GQ_API gq_status gq_gemv_q4_0_grouped(const gq_gemv_desc* mats, int count, int64_t K,
+                                      const void* x, int x_dtype, int64_t B, int y_dtype,
+                                      unsigned flags, int* dev_status, void* stream) {
+  return gq::gemv_grouped_entry<GQ_FMT_Q4_0>(mats, count, K, x, x_dtype, B, y_dtype, flags,
+                                             dev_status, stream);
+}
+
+GQ_API gq_status gq_gemv_ksb_grouped(const gq_gemv_desc* mats, int count, int64_t K,
+                                     const void* x, int x_dtype, int64_t B, int y_dtype,
+                                     unsigned flags, int* dev_status, void* stream) {
+  return gq::gemv_grouped_entry<GQ_FMT_KSB>(mats, count, K, x, x_dtype, B, y_dtype, flags,
+                                            dev_status, stream);
 }
 
 // Allocation-free batch-1 Q4_0 GEMV: the integer tensor-core path of

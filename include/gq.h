@@ -183,6 +183,34 @@ GQ_API gq_status gq_gemv_ksb(const void* W, int64_t M, int64_t K,
                              void* y, int y_dtype, void* workspace, size_t ws_bytes,
                              unsigned flags, int* dev_status, void* stream);
 
+/* Grouped dequantize-fused GEMV: several matrices that share K and the
+ * activations, y_i[b][m] = sum_k W_hat_i[m][k] * x[b][k] for every descriptor
+ * (the same operation as gq_gemv_q4_0 / gq_gemv_ksb, matrix by matrix).  It
+ * serves a decode step that multiplies one activation vector by many weight
+ * matrices: the whole-model stream, or the projections that read the same x.
+ * The pages stream one matrix at a time; this entry point has no counterpart
+ * on them.  One launch covers up to 256 matrices: its CTAs load x once and
+ * stream the 16-row groups of all of them back to back, so there is no
+ * launch gap and no repeated activation load between matrices.
+ *   mats:  count host descriptors {W, M, y} (read during the call only).  W as
+ *          for gq_gemv_*, 16-byte aligned; y: [B][M] of y_dtype, 16-byte
+ *          aligned.  M == 0 entries are skipped (W and y may then be NULL).
+ *   K, x, x_dtype, B, y_dtype, flags, dev_status: as for gq_gemv_*, shared by
+ *          all matrices (the integer path and its workspace do not apply).
+ * Validation covers every descriptor before anything is launched; more than
+ * 256 matrices are processed in several launches in stream order. */
+typedef struct gq_gemv_desc {
+    const void* W;
+    int64_t M;
+    void* y;
+} gq_gemv_desc;
+GQ_API gq_status gq_gemv_q4_0_grouped(const gq_gemv_desc* mats, int count, int64_t K,
+                                      const void* x, int x_dtype, int64_t B, int y_dtype,
+                                      unsigned flags, int* dev_status, void* stream);
+GQ_API gq_status gq_gemv_ksb_grouped(const gq_gemv_desc* mats, int count, int64_t K,
+                                     const void* x, int x_dtype, int64_t B, int y_dtype,
+                                     unsigned flags, int* dev_status, void* stream);
+
 /* Allocation-free variant (no counterpart on the pages): the batch-1 integer
  * tensor-core path of gq_gemv_q4_0 (fp16 x, B = 1) with its scratch -- the
  * per-CTA counts and partial sums, 33 KB -- in a static device array of the

@@ -121,6 +121,37 @@ def test_gemv_validation(name, block):
     assert call(st=A + 2) == ALIGN
 
 
+def test_gemv_grouped_validation():
+    import ctypes
+    D = gq.GemvDesc
+    for name in ("gq_gemv_q4_0_grouped", "gq_gemv_ksb_grouped"):
+        f = getattr(gq.lib, name)
+        K = 256
+
+        def call(descs, count=None, K=K, x=A, xt=1, B=1, yt=1, flags=0, st=None):
+            arr = (D * max(len(descs), 1))(*descs)
+            n = len(descs) if count is None else count
+            return f(ctypes.cast(arr, ctypes.c_void_p), n, K, x, xt, B, yt, flags, st, None)
+
+        good = D(A, 16, A + 4096)
+        assert call([good], count=-1) == INVALID
+        assert f(None, 1, K, A, 1, 1, 1, 0, None, None) == INVALID
+        assert call([D(A, -1, A)]) == INVALID
+        assert call([good, D(A + 2, 16, A)]) == ALIGN           # every descriptor is checked
+        assert call([good, D(A, 16, A + 8)]) == ALIGN
+        assert call([good, D(None, 16, A)]) == INVALID
+        assert call([good, D(A, 16, None)]) == INVALID
+        assert call([good], K=K + 16) == SHAPE
+        assert call([good], B=9) == SHAPE
+        assert call([good], xt=7) == DTYPE and call([good], yt=7) == DTYPE
+        assert call([good], flags=2) == INVALID
+        assert call([good], x=None) == INVALID and call([good], x=A + 2) == ALIGN
+        assert call([good], st=A + 2) == ALIGN
+        assert call([], count=0) == GQ_OK                      # nothing to do: no launch
+        assert call([D(None, 0, None), D(None, 0, None)]) == GQ_OK
+        assert call([good], B=0) == GQ_OK
+
+
 def test_binding_refuses_host_tensors():
     import torch
     with pytest.raises(ValueError):

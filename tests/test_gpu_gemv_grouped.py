@@ -1,0 +1,99 @@
+"""Grouped GEMV (gq_gemv_*_grouped): several matrices sharing K and x in one
+launch.  Every output is compared with the oracle's fp64 product (tolerance as
+in test_gpu_gemv.py) and with the single-matrix entry point, which computes
+each row with the same arithmetic in the same order, so the two agree bit for
+bit."""
+import numpy as np
+import pytest
+import torch
+
+import bit_gemv_q4_b200 as gq
+import oracle
+import synth
+from gpu_helpers import KSB, Q40, assert_product_close, x_for_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+def _mats(fmt, Ms, K, seed):
+    qs = []
+    for i, M in enumerate(Ms):
+        if M == 0:
+            qs.append(np.zeros(0, np.uint8))
+            continue
+        w = synth.gaussian_weights(M, K, seed=seed + i).numpy().ravel()
+        q, _ = oracle.quantize(fmt, w)
+        qs.append(q)
+    return qs
+
+
+def _grouped(fmt, Wd, Ms, K, x, ydt, flags=0):
+    f = gq.gq_gemv_q4_0_grouped if fmt == Q40 else gq.gq_gemv_ksb_grouped
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    outs = f(Wd, Ms, K, x, y_dtype=ydt, flags=flags, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    return outs
+
+
+def _single(fmt, W, M, K, x, ydt):
+    f = gq.gq_gemv_q4_0 if fmt == Q40 else gq.gq_gemv_ksb
+    y = f(W, M, K, x, y_dtype=ydt)
+    torch.cuda.synchronize()
+    return y
+
+
+@pytest.mark.parametrize("fmt,K,B,xdt,ydt", [
+    (Q40, 4096, 1, torch.float16, torch.float16),
+    (Q40, 2080, 3, torch.bfloat16, torch.float32),   # ragged chunks, unaligned rows
+    (KSB, 4096, 1, torch.float16, torch.float16),
+    (KSB, 2304, 2, torch.float32, torch.bfloat16),
+])
+def test_grouped_matches_oracle_and_single(fmt, K, B, xdt, ydt):
+    Ms = [4096, 17, 0, 1, 300, 33, 2048]
+    qs = _mats(fmt, Ms, K, seed=100 + K)
+    Wd = [torch.from_numpy(q).cuda() if q.size else None for q in qs]
+    x = synth.activations(B, K, seed=5, dtype=xdt).cuda()
+    outs = _grouped(fmt, Wd, Ms, K, x, ydt)
+    xo, xt = x_for_oracle(x)
+    for q, W, M, y in zip(qs, Wd, Ms, outs):
+        assert tuple(y.shape) == (B, M)
+        if M == 0:
+            continue
+        Y, bound = oracle.gemm(fmt, q, M, K, xo, xt)
+        assert_product_close(y, Y, bound)
+        ys = _single(fmt, W, M, K, x, ydt)
+        assert torch.equal(y.view(torch.int16) if y.dtype != torch.float32 else y.view(torch.int32),
+                           ys.view(torch.int16) if ys.dtype != torch.float32 else ys.view(torch.int32))
+
+
+def test_grouped_more_matrices_than_one_launch():
+    # 300 matrices (more than one launch's table), with PDL between launches
+    K = 512
+    Ms = [(i * 37) % 70 + 1 for i in range(300)]
+    qs = _mats(Q40, Ms, K, seed=7)
+    Wd = [torch.from_numpy(q).cuda() for q in qs]
+    x = synth.activations(1, K, seed=3, dtype=torch.float16).cuda()
+    outs = _grouped(Q40, Wd, Ms, K, x, torch.float16, flags=gq.GQ_GEMV_PDL)
+    xo, xt = x_for_oracle(x)
+    for q, M, y in zip(qs, Ms, outs):
+        Y, bound = oracle.gemm(Q40, q, M, K, xo, xt)
+        assert_product_close(y, Y, bound)
+
+
+def test_grouped_model_layer_shapes():
+    # one decoder layer of the whole-model stream: 4 x 4096^2 and 3 x 11008x4096,
+    # one x; checked against the single-matrix calls
+    K = 4096
+    Ms = [4096, 4096, 4096, 4096, 11008, 11008, 4096]
+    rng_seeds = 30000
+    Wd, ys = [], []
+    x = synth.activations(1, K, seed=9, dtype=torch.float16).cuda()
+    for i, M in enumerate(Ms):
+        w = synth.gaussian_weights(M, K, seed=rng_seeds + i, device="cuda")
+        W = gq.gq_quantize_q4_0(w.view(-1))
+        Wd.append(W)
+        ys.append(_single(Q40, W, M, K, x, torch.float16))
+    outs = _grouped(Q40, Wd, Ms, K, x, torch.float16, flags=gq.GQ_GEMV_PDL)
+    for y, ys_ in zip(outs, ys):
+        assert torch.equal(y.view(torch.int16), ys_.view(torch.int16))
