@@ -35,13 +35,13 @@ METRIC = "Q4 GEMV streamed-weight GB/s and % of HBM peak (4096x11008, batch 1)"
 CASES = [("q4_0", 4096, 11008), ("q4_0", 11008, 4096), ("ksb", 4096, 11008), ("ksb", 11008, 4096)]
 FALLBACK_HBM_GBS = 6650.0
 
-# DRAM bytes per GEMV launch (mean over the four cases) from one ncu capture
-# (profiles/gemv_q4_0_4096x11008.md).  Reported only while the GEMV sources
-# hash to what was profiled; any change to the kernel makes it null.
+# DRAM bytes (read + write) of one GEMV launch, the q4_0 4096x11008 case, from
+# one ncu capture (profiles/gemv_q4_0_4096x11008.md).  Reported only while the
+# GEMV sources hash to what was profiled; any change to the kernel makes it null.
 GEMV_TRAFFIC = {
-    "bytes": 25407744,
+    "bytes": 25406976,
     "sources": {
-        "bit_gemv_q4_b200/csrc/gq_gemv.cu": "3a396a231f0b52d94bea082f9ba47776c70c402d1dd37454c481e99a3489e87c",
+        "bit_gemv_q4_b200/csrc/gq_gemv.cu": "5e85c2817fc4593121c080f87507f15029f12fca99c6d275509617e1374c08fd",
         "bit_gemv_q4_b200/csrc/gq_device.cuh": "c88e136b756c0355212db717041e37b38523df1a913fe4fa63cd047c2a12e5f4",
     },
 }
@@ -577,14 +577,49 @@ def run_suite(path):
 
 
 def run_single(spec, launches, batch, flags, use_ws=False):
-    """A few launches of one product on distinct copies of one matrix (for
-    profilers): spec = "gemv:q4_0:4096:11008" or "gemm:ksb:11008:4096"."""
+    """A few launches of one hot-path call (for profilers).  spec:
+    "gemv:q4_0:4096:11008" / "gemm:ksb:11008:4096" (distinct copies of one
+    matrix), "grouped:q4_0:<layers>" (the decoder-layer matrices
+    4 x 4096x4096 + 3 x 11008x4096 per layer in one grouped call), or
+    "quantize:ksb:<n>" / "dequantize:q4_0:<n>" (n weights)."""
     import torch
     import bit_gemv_q4_b200 as gq
     import synth
-    kind, fmt, M, K = spec.split(":")
-    M, K = int(M), int(K)
     dev = torch.device("cuda", torch.cuda.current_device())
+    parts = spec.split(":")
+    if parts[0] == "grouped":
+        fmt, layers = parts[1], int(parts[2])
+        quant = gq.gq_quantize_q4_0 if fmt == "q4_0" else gq.gq_quantize_ksb
+        Ms = ([4096] * 4 + [11008] * 3) * layers
+        Ws, nb = [], 0
+        for i, M in enumerate(Ms):
+            w = synth.gaussian_weights(M, 4096, seed=30000 + i, device=dev)
+            Ws.append(quant(w.view(-1)))
+            nb += Ws[-1].numel()
+            del w
+        x = synth.activations(batch, 4096, seed=9, dtype=torch.float16, device=dev)
+        outs = [torch.empty((batch, M), dtype=torch.float16, device=dev) for M in Ms]
+        fg = gq.gq_gemv_q4_0_grouped if fmt == "q4_0" else gq.gq_gemv_ksb_grouped
+        for _ in range(launches):
+            fg(Ws, Ms, 4096, x, outs=outs, flags=flags)
+        torch.cuda.synchronize()
+        print(json.dumps({"single": spec, "batch": batch, "launches": launches, "bytes": nb}))
+        return
+    if parts[0] in ("quantize", "dequantize"):
+        fmt, n = parts[1], int(parts[2])
+        x = torch.randn(n, device=dev, dtype=torch.float32)
+        qf = gq.gq_quantize_q4_0 if fmt == "q4_0" else gq.gq_quantize_ksb
+        q = qf(x)
+        for _ in range(launches):
+            if parts[0] == "quantize":
+                qf(x, out=q)
+            else:
+                (gq.gq_dequantize_q4_0 if fmt == "q4_0" else gq.gq_dequantize_ksb)(q, n, out=x)
+        torch.cuda.synchronize()
+        print(json.dumps({"single": spec, "launches": launches, "bytes": q.numel() + 4 * n}))
+        return
+    kind, fmt, M, K = parts
+    M, K = int(M), int(K)
     w = synth.gaussian_weights(M, K, seed=1, device=dev)
     q = (gq.gq_quantize_q4_0 if fmt == "q4_0" else gq.gq_quantize_ksb)(w.view(-1))
     del w
@@ -621,7 +656,8 @@ def main():
     ap.add_argument("--suite", default=None,
                     help="also measure every hot-path row; JSON lines written to this file")
     ap.add_argument("--single", default=None,
-                    help="profiling aid: launch one product a few times, e.g. gemv:q4_0:4096:11008")
+                    help="profiling aid: launch one call a few times, e.g. gemv:q4_0:4096:11008, "
+                         "grouped:q4_0:2, quantize:ksb:268435456")
     ap.add_argument("--launches", type=int, default=4)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--flags", type=int, default=0)
