@@ -45,6 +45,7 @@
 
 #include "gq.h"
 #include "gq_device.cuh"
+#include "gq_gemv.h"
 #include "gq_host.h"
 #include "gq_tc.cuh"
 
@@ -689,6 +690,10 @@ gq_status gemm_entry(const void* W, int64_t M, int64_t K, const void* X, int xt,
   const size_t need = gemm_ws_bytes(M, K, N, &parts_off);
   if (!workspace || ws_bytes < need) return GQ_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return GQ_ERR_ALIGNMENT;
+  // narrow batches: the warp-MMA product (every weight decoded once for all
+  // columns, no tcgen05 instruction per 16 columns)
+  if (B <= kWarpMmaMaxB)
+    return gemv_batched(FMT, W, M, K, X, xt, B, Y, yt, dev_status, as_stream(stream));
 
   EncodeTiled enc = tensor_map_encoder();
   if (!enc) return GQ_ERR_CUDA;

@@ -41,6 +41,7 @@
 
 #include "gq.h"
 #include "gq_device.cuh"
+#include "gq_gemv.h"
 #include "gq_gemv_i8.h"
 #include "gq_host.h"
 
@@ -73,7 +74,15 @@ constexpr int kStageBytes = kRows * kPitch + 16;    // +16: window-read slack
 constexpr int kStages = GQ_GEMV_STAGES;
 constexpr int kXBlk = 64;                           // B-fragment bytes per 32 weights
 constexpr int kXStride = (kChunkW / 32) * kXBlk + 64;  // per (chunk, batch row), padded
-constexpr int kRedBytes = 2 * kConsumers * 32 * 4 * 4;  // cross-warp reduction
+// The batch occupies NT n8 tiles of the MMA's N dimension: NT = 0 is one
+// activation vector (with its own fragment layout, x_frag), NT = 1 covers
+// B <= 8 and NT = 2 covers B <= 16.  Fragments and accumulators hold four
+// floats per tile.
+constexpr int acc_len(int nt) { return 4 * (nt > 1 ? nt : 1); }
+constexpr int kMaxNT = 2;
+// cross-warp reduction buffer of a launch with NT tiles (two groups in flight)
+constexpr int red_bytes(int nt) { return 2 * kConsumers * 32 * acc_len(nt) * 4; }
+constexpr int kRedBytes = red_bytes(kMaxNT);  // the largest
 // activation window budget: what the stages and the reduction leave of the
 // 227 KB a CTA may hold, at most 72 KB
 constexpr int kXSmemFree = 227 * 1024 - kStages * kStageBytes - kRedBytes - 1024;
@@ -83,6 +92,7 @@ static_assert(kChunkW == 1024 || kChunkW == 2048, "supported chunk sizes");
 static_assert(kSubPerWarp % 2 == 0, "blocks per warp come in pairs");
 
 enum { XT_F16 = 0, XT_BF16 = 1, XT_F32 = 2 };
+
 
 template <int FMT>
 struct Fmt;
@@ -219,9 +229,9 @@ __device__ __forceinline__ uint32_t ld32_even(uint32_t off) {
 // zeros): the shared-memory load then touches 2 of the warp's 8 lane
 // quarters, and columns 0 and 2 of the result put row r in lane t = 0 and
 // row r+8 in lane t = 1.
-template <bool NB1>
+template <int NT>
 __device__ __forceinline__ uint4 x_frag(uint32_t xp) {
-  if constexpr (NB1) {
+  if constexpr (NT == 0) {
     const int lane = threadIdx.x & 31;
     return (lane & 0x14) == 0 ? ld128(xp) : make_uint4(0u, 0u, 0u, 0u);
   } else {
@@ -230,29 +240,38 @@ __device__ __forceinline__ uint4 x_frag(uint32_t xp) {
 }
 
 // One 32-weight block for rows r (codes qa) and r+8 (codes qb): both k16
-// MMAs over every activation term, into a fresh fragment c.
-template <int XT, bool NB1>
-__device__ __forceinline__ void block_mma(float c[4], uint32_t qa, uint32_t qb, uint32_t xp,
-                                          uint32_t term_stride) {
+// MMAs over every activation term and every n8 tile, into a fresh fragment c
+// (tile n in c[4n..4n+3]).  The codes are decoded once for all tiles; tile 1
+// reads the batch row xt1 bytes past tile 0's.
+template <int XT, int NT>
+__device__ __forceinline__ void block_mma(float* c, uint32_t qa, uint32_t qb, uint32_t xp,
+                                          uint32_t term_stride, uint32_t xt1) {
   constexpr int kTerms = (XT == XT_F32) ? 3 : 1;
+  constexpr int kTiles = NT > 1 ? NT : 1;
   uint32_t ra[4], rb[4];
   if constexpr (XT == XT_F16) {
     decode_f16(qa, ra);
     decode_f16(qb, rb);
-    const uint4 xv = x_frag<NB1>(xp);
-    mma_f16_z(c, ra[0], rb[0], ra[2], rb[2], xv.x, xv.y);
-    mma_f16(c, ra[1], rb[1], ra[3], rb[3], xv.z, xv.w);
+#pragma unroll
+    for (int n = 0; n < kTiles; ++n) {
+      const uint4 xv = x_frag<NT>(xp + n * xt1);
+      mma_f16_z(c + 4 * n, ra[0], rb[0], ra[2], rb[2], xv.x, xv.y);
+      mma_f16(c + 4 * n, ra[1], rb[1], ra[3], rb[3], xv.z, xv.w);
+    }
   } else {
     decode_bf16(qa, ra);
     decode_bf16(qb, rb);
 #pragma unroll
-    for (int tm = 0; tm < kTerms; ++tm) {
-      const uint4 xv = x_frag<NB1>(xp + tm * term_stride);
-      if (tm == 0)
-        mma_bf16_z(c, ra[0], rb[0], ra[2], rb[2], xv.x, xv.y);
-      else
-        mma_bf16(c, ra[0], rb[0], ra[2], rb[2], xv.x, xv.y);
-      mma_bf16(c, ra[1], rb[1], ra[3], rb[3], xv.z, xv.w);
+    for (int n = 0; n < kTiles; ++n) {
+#pragma unroll
+      for (int tm = 0; tm < kTerms; ++tm) {
+        const uint4 xv = x_frag<NT>(xp + n * xt1 + tm * term_stride);
+        if (tm == 0)
+          mma_bf16_z(c + 4 * n, ra[0], rb[0], ra[2], rb[2], xv.x, xv.y);
+        else
+          mma_bf16(c + 4 * n, ra[0], rb[0], ra[2], rb[2], xv.x, xv.y);
+        mma_bf16(c + 4 * n, ra[1], rb[1], ra[3], rb[3], xv.z, xv.w);
+      }
     }
   }
 }
@@ -261,23 +280,26 @@ __device__ __forceinline__ void block_mma(float c[4], uint32_t qa, uint32_t qb, 
 // activation vector (x_frag) lane t = 0 keeps row r (c[0], column 0) and
 // lane t = 1 row r+8 (c[2], column 2), each in acc[0] with its own row's
 // scale d0; lanes t = 2, 3 accumulate zeros.
-template <bool NB1>
-__device__ __forceinline__ void scale_acc(float acc[4], const float c[4], float d0, float d1) {
-  if constexpr (NB1) {
+template <int NT>
+__device__ __forceinline__ void scale_acc(float* acc, const float* c, float d0, float d1) {
+  if constexpr (NT == 0) {
     const int t = threadIdx.x & 3;
     acc[0] = fmaf(d0, (t & 1) ? c[2] : c[0], acc[0]);
   } else {
-    acc[0] = fmaf(d0, c[0], acc[0]);
-    acc[2] = fmaf(d1, c[2], acc[2]);
-    acc[1] = fmaf(d0, c[1], acc[1]);
-    acc[3] = fmaf(d1, c[3], acc[3]);
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      acc[4 * n + 0] = fmaf(d0, c[4 * n + 0], acc[4 * n + 0]);
+      acc[4 * n + 2] = fmaf(d1, c[4 * n + 2], acc[4 * n + 2]);
+      acc[4 * n + 1] = fmaf(d0, c[4 * n + 1], acc[4 * n + 1]);
+      acc[4 * n + 3] = fmaf(d1, c[4 * n + 3], acc[4 * n + 3]);
+    }
   }
 }
 
 // ---------------------------------------------------------------- Q4_0 body
 // Block j of a stage: its two rows' code words and scales (with one
 // activation vector only the scale of this lane's output row, at rowd).
-template <bool ALIGNED, int J, bool NB1>
+template <bool ALIGNED, int J, int NT>
 __device__ __forceinline__ void q40_load(uint32_t row0, uint32_t row1, uint32_t rowd, int t,
                                          int jb, uint32_t& qa, uint32_t& qb, float& da,
                                          float& db) {
@@ -292,7 +314,7 @@ __device__ __forceinline__ void q40_load(uint32_t row0, uint32_t row1, uint32_t 
     qa = ld32_even(a + 2 + 4 * t);
     qb = ld32_even(b + 2 + 4 * t);
   }
-  if constexpr (NB1) {
+  if constexpr (NT == 0) {
     da = half_bits_to_float(ld16(rowd + jb * 18));
     db = da;
   } else {
@@ -304,9 +326,9 @@ __device__ __forceinline__ void q40_load(uint32_t row0, uint32_t row1, uint32_t 
 // A consumer warp's blocks w*kSubPerWarp .. +kSubPerWarp-1 of one stage.  A
 // full share is unrolled without branches -- every load is issued before the
 // first decode -- so the warp keeps many loads and MMAs in flight.
-template <int XT, bool NB1, bool ALIGNED>
-__device__ __forceinline__ void q40_chunk(float acc[4], uint32_t row0, uint32_t row1,
-                                          uint32_t xw, uint32_t term_stride, int w, int t,
+template <int XT, int NT, bool ALIGNED>
+__device__ __forceinline__ void q40_chunk(float* acc, uint32_t row0, uint32_t row1, uint32_t xw,
+                                          uint32_t term_stride, uint32_t xt1, int w, int t,
                                           int nvalid) {
   const int jw = w * kSubPerWarp;  // even
   const uint32_t rowd = (t & 1) ? row1 : row0;
@@ -315,25 +337,25 @@ __device__ __forceinline__ void q40_chunk(float acc[4], uint32_t row0, uint32_t 
     float da[kSubPerWarp], db[kSubPerWarp];
 #pragma unroll
     for (int j = 0; j < kSubPerWarp; j += 2) {
-      q40_load<ALIGNED, 0, NB1>(row0, row1, rowd, t, jw + j, qa[j], qb[j], da[j], db[j]);
-      q40_load<ALIGNED, 1, NB1>(row0, row1, rowd, t, jw + j + 1, qa[j + 1], qb[j + 1], da[j + 1],
-                                db[j + 1]);
+      q40_load<ALIGNED, 0, NT>(row0, row1, rowd, t, jw + j, qa[j], qb[j], da[j], db[j]);
+      q40_load<ALIGNED, 1, NT>(row0, row1, rowd, t, jw + j + 1, qa[j + 1], qb[j + 1], da[j + 1],
+                               db[j + 1]);
     }
 #pragma unroll
     for (int j = 0; j < kSubPerWarp; ++j) {
-      float c[4];
-      block_mma<XT, NB1>(c, qa[j], qb[j], xw + (jw + j) * kXBlk, term_stride);
-      scale_acc<NB1>(acc, c, da[j], db[j]);
+      float c[acc_len(NT)];
+      block_mma<XT, NT>(c, qa[j], qb[j], xw + (jw + j) * kXBlk, term_stride, xt1);
+      scale_acc<NT>(acc, c, da[j], db[j]);
     }
   } else {
     // ragged last chunk of a row
     for (int j = 0; j < nvalid; ++j) {
       uint32_t qa, qb;
       float da, db;
-      q40_load<false, 0, NB1>(row0, row1, rowd, t, jw + j, qa, qb, da, db);
-      float c[4];
-      block_mma<XT, NB1>(c, qa, qb, xw + (jw + j) * kXBlk, term_stride);
-      scale_acc<NB1>(acc, c, da, db);
+      q40_load<false, 0, NT>(row0, row1, rowd, t, jw + j, qa, qb, da, db);
+      float c[acc_len(NT)];
+      block_mma<XT, NT>(c, qa, qb, xw + (jw + j) * kXBlk, term_stride, xt1);
+      scale_acc<NT>(acc, c, da, db);
     }
   }
 }
@@ -342,25 +364,28 @@ __device__ __forceinline__ void q40_chunk(float acc[4], uint32_t row0, uint32_t 
 // A consumer warp's kSubPerWarp sub-blocks of one super-block of the stage.
 // s~_j = S * q_j is applied as q_j per sub-block and S once at the end.  All
 // loads are issued before the first decode.
-template <int XT, bool NB1>
-__device__ __forceinline__ void ksb_chunk(float acc[4], uint32_t row0, uint32_t row1,
-                                          uint32_t xw, uint32_t term_stride, int w, int t) {
+template <int XT, int NT>
+__device__ __forceinline__ void ksb_chunk(float* acc, uint32_t row0, uint32_t row1, uint32_t xw,
+                                          uint32_t term_stride, uint32_t xt1, int w, int t) {
+  constexpr bool kOne = (NT == 0);
   const int sb = (w * kSubPerWarp) >> 3, j0 = (w * kSubPerWarp) & 7;
   const uint32_t a = row0 + sb * 138;
   const uint32_t b = row1 + sb * 138;
   // scales of rows r and r+8; with one activation vector only this lane's
   // output row (scale_acc), read into both
-  const uint32_t sa = NB1 ? ((t & 1) ? b : a) : a;
+  const uint32_t sa = kOne ? ((t & 1) ? b : a) : a;
   const float Sa = half_bits_to_float(ld16(sa));
-  const float Sb = NB1 ? Sa : half_bits_to_float(ld16(b));
+  const float Sb = kOne ? Sa : half_bits_to_float(ld16(b));
   uint32_t qja[2], qjb[2];
   qja[0] = ld32_even(sa + 2 + j0);
-  qjb[0] = NB1 ? qja[0] : ld32_even(b + 2 + j0);
+  qjb[0] = kOne ? qja[0] : ld32_even(b + 2 + j0);
   if constexpr (kSubPerWarp > 4) {
     qja[1] = ld32_even(sa + 6 + j0);
-    qjb[1] = NB1 ? qja[1] : ld32_even(b + 6 + j0);
+    qjb[1] = kOne ? qja[1] : ld32_even(b + 6 + j0);
   }
-  float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+  float sacc[acc_len(NT)];
+#pragma unroll
+  for (int i = 0; i < acc_len(NT); ++i) sacc[i] = 0.f;
   constexpr int kBatch = kSubPerWarp < 4 ? kSubPerWarp : 4;
 #pragma unroll
   for (int h = 0; h < kSubPerWarp; h += kBatch) {  // batches of up to four sub-blocks
@@ -372,19 +397,24 @@ __device__ __forceinline__ void ksb_chunk(float acc[4], uint32_t row0, uint32_t 
     }
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
-      float c[4];
-      block_mma<XT, NB1>(c, na[j], nb[j], xw + (8 * sb + j0 + h + j) * kXBlk, term_stride);
+      float c[acc_len(NT)];
+      block_mma<XT, NT>(c, na[j], nb[j], xw + (8 * sb + j0 + h + j) * kXBlk, term_stride, xt1);
       const int q = h + j;  // sub-block index within this warp's share
       const float fa = static_cast<float>(static_cast<int8_t>((qja[q >> 2] >> (8 * (q & 3))) & 0xFFu));
       const float fb = static_cast<float>(static_cast<int8_t>((qjb[q >> 2] >> (8 * (q & 3))) & 0xFFu));
-      scale_acc<NB1>(sacc, c, fa, fb);
+      scale_acc<NT>(sacc, c, fa, fb);
     }
   }
-  acc[0] = fmaf(Sa, sacc[0], acc[0]);
-  if constexpr (!NB1) {
-    acc[2] = fmaf(Sb, sacc[2], acc[2]);
-    acc[1] = fmaf(Sa, sacc[1], acc[1]);
-    acc[3] = fmaf(Sb, sacc[3], acc[3]);
+  if constexpr (kOne) {
+    acc[0] = fmaf(Sa, sacc[0], acc[0]);
+  } else {
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      acc[4 * n + 0] = fmaf(Sa, sacc[4 * n + 0], acc[4 * n + 0]);
+      acc[4 * n + 1] = fmaf(Sa, sacc[4 * n + 1], acc[4 * n + 1]);
+      acc[4 * n + 2] = fmaf(Sb, sacc[4 * n + 2], acc[4 * n + 2]);
+      acc[4 * n + 3] = fmaf(Sb, sacc[4 * n + 3], acc[4 * n + 3]);
+    }
   }
 }
 
@@ -476,7 +506,7 @@ __device__ void load_x_window(uint8_t* xs, const void* x, int64_t K, int B, int 
   }
 }
 
-template <int FMT, int XT, bool NB1, bool ALIGNED, class Tbl>
+template <int FMT, int XT, int NT, bool ALIGNED, class Tbl>
 __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
     gemv_kernel(const GemvArgs a, const __grid_constant__ Tbl tbl) {
   constexpr int kBlkW = Fmt<FMT>::kBlkW, kBlkB = Fmt<FMT>::kBlkB;
@@ -487,8 +517,9 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
   uint8_t* stages = smem;
   uint8_t* xs = smem + kStages * kStageBytes;
   const uint32_t term_stride = static_cast<uint32_t>(a.win * a.B * kXStride);
-  float* red = reinterpret_cast<float*>(xs + kTerms * term_stride);  // [2][kConsumers][32][4]
-  uint64_t* full = reinterpret_cast<uint64_t*>(red + 2 * kConsumers * 32 * 4);
+  // [2][kConsumers][32][acc_len(NT)]
+  float* red = reinterpret_cast<float*>(xs + kTerms * term_stride);
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + 2 * kConsumers * 32 * acc_len(NT));
   uint64_t* empty = full + kStages;
   uint64_t* cbar = empty + kStages;  // consumer-group barrier (bounded waits)
   int* abort_flag = reinterpret_cast<int*>(cbar + 1);
@@ -609,6 +640,8 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
   }
   const uint32_t x_chunk = static_cast<uint32_t>(a.B * kXStride);
   const uint32_t x_lane = static_cast<uint32_t>(xs - smem) + bsel * kXStride + t * 16;
+  // n8 tile 1 holds batch rows 8..15: this lane's row there, relative to tile 0
+  const uint32_t xt1 = static_cast<uint32_t>((min(8 + r, a.B - 1) - bsel) * kXStride);
 
   int s = 0;        // stage of the next use
   uint32_t ph = 0;  // its phase parity
@@ -617,7 +650,9 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
   for (int g = blockIdx.x; g < a.ngroups && ok; g += gridDim.x, ++gi) {
     const Unit un = unit_of(a, tbl, g, cmi);
     const int64_t m0 = un.m0;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float acc[acc_len(NT)];
+#pragma unroll
+    for (int q = 0; q < acc_len(NT); ++q) acc[q] = 0.f;
     // offset of row r's (and r+8's) first byte inside its 16-byte granule
     uint32_t off0 = static_cast<uint32_t>(
         (reinterpret_cast<uintptr_t>(un.W) + static_cast<uintptr_t>((m0 + r) * a.rowbytes)) & 15u);
@@ -642,16 +677,16 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
       if constexpr (FMT == GQ_FMT_Q4_0) {
         const int nvalid = whole ? kSubPerWarp : tail_valid;
         if constexpr (ALIGNED) {
-          q40_chunk<XT, NB1, true>(acc, stg + r * kPitch, stg + (r + 8) * kPitch, xw,
-                                   term_stride, cw, t, nvalid);
+          q40_chunk<XT, NT, true>(acc, stg + r * kPitch, stg + (r + 8) * kPitch, xw,
+                                  term_stride, xt1, cw, t, nvalid);
         } else {
-          q40_chunk<XT, NB1, false>(acc, stg + r * kPitch + off0, stg + (r + 8) * kPitch + off1,
-                                    xw, term_stride, cw, t, nvalid);
+          q40_chunk<XT, NT, false>(acc, stg + r * kPitch + off0, stg + (r + 8) * kPitch + off1,
+                                   xw, term_stride, xt1, cw, t, nvalid);
         }
       } else {
         if (whole || tail_valid)
-          ksb_chunk<XT, NB1>(acc, stg + r * kPitch + off0, stg + (r + 8) * kPitch + off1, xw,
-                             term_stride, cw, t);
+          ksb_chunk<XT, NT>(acc, stg + r * kPitch + off0, stg + (r + 8) * kPitch + off1, xw,
+                            term_stride, xt1, cw, t);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
@@ -668,31 +703,43 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
 
     // reduce the consumer warps' partial sums (double-buffered by group
     // parity, so one barrier per group suffices), then store
-    float* rb = red + (gi & 1) * kConsumers * 32 * 4;
-    reinterpret_cast<float4*>(rb)[cw * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    constexpr int kTiles = NT > 1 ? NT : 1;
+    float4* rb = reinterpret_cast<float4*>(red) + (gi & 1) * kConsumers * 32 * kTiles;
+#pragma unroll
+    for (int n = 0; n < kTiles; ++n)
+      rb[(cw * 32 + lane) * kTiles + n] =
+          make_float4(acc[4 * n], acc[4 * n + 1], acc[4 * n + 2], acc[4 * n + 3]);
     if (!group_sync()) { ok = false; break; }
     if (cw == 0) {
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      float s4[acc_len(NT)];
+#pragma unroll
+      for (int q = 0; q < acc_len(NT); ++q) s4[q] = 0.f;
 #pragma unroll
       for (int w = 0; w < kConsumers; ++w) {
-        const float4 v = reinterpret_cast<const float4*>(rb)[w * 32 + lane];
-        s4[0] += v.x;
-        s4[1] += v.y;
-        s4[2] += v.z;
-        s4[3] += v.w;
+#pragma unroll
+        for (int n = 0; n < kTiles; ++n) {
+          const float4 v = rb[(w * 32 + lane) * kTiles + n];
+          s4[4 * n + 0] += v.x;
+          s4[4 * n + 1] += v.y;
+          s4[4 * n + 2] += v.z;
+          s4[4 * n + 3] += v.w;
+        }
       }
       const int64_t ra = m0 + r, rbw = m0 + r + 8;
-      if (NB1) {
+      if constexpr (NT == 0) {
         // lane t = 0 holds row r, lane t = 1 row r + 8 (scale_acc)
         const int64_t row = (t == 0) ? ra : rbw;
         if (t < 2 && row < un.M) store_elem(un.y, row, s4[0], a.ytype);
       } else {
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int col = 2 * t + i;
-          if (col < a.B) {
-            if (ra < un.M) store_elem(un.y, col * un.M + ra, s4[i], a.ytype);
-            if (rbw < un.M) store_elem(un.y, col * un.M + rbw, s4[2 + i], a.ytype);
+        for (int n = 0; n < kTiles; ++n) {
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int col = 8 * n + 2 * t + i;
+            if (col < a.B) {
+              if (ra < un.M) store_elem(un.y, col * un.M + ra, s4[4 * n + i], a.ytype);
+              if (rbw < un.M) store_elem(un.y, col * un.M + rbw, s4[4 * n + 2 + i], a.ytype);
+            }
           }
         }
       }
@@ -706,15 +753,16 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
 }
 
 size_t gemv_smem_bytes(int B, int terms, int win) {
+  const int nt = B == 1 ? 0 : (B <= 8 ? 1 : 2);
   return static_cast<size_t>(kStages) * kStageBytes +
-         static_cast<size_t>(terms) * win * B * kXStride + kRedBytes +
+         static_cast<size_t>(terms) * win * B * kXStride + red_bytes(nt) +
          (2 * kStages + 1) * sizeof(uint64_t) + 16;
 }
 
-template <int FMT, int XT, bool NB1, bool ALIGNED, class Tbl>
+template <int FMT, int XT, int NT, bool ALIGNED, class Tbl>
 gq_status launch_gemv(const GemvArgs& a, const Tbl& tbl, cudaStream_t stream, bool pdl) {
   constexpr int kTerms = (XT == XT_F32) ? 3 : 1;
-  auto kern = gemv_kernel<FMT, XT, NB1, ALIGNED, Tbl>;
+  auto kern = gemv_kernel<FMT, XT, NT, ALIGNED, Tbl>;
   const size_t smem = gemv_smem_bytes(a.B, kTerms, a.win);
   static int configured_dev = -1;
   static size_t configured_smem = 0;
@@ -751,14 +799,17 @@ gq_status launch_gemv(const GemvArgs& a, const Tbl& tbl, cudaStream_t stream, bo
 template <int FMT, int XT, class Tbl>
 gq_status dispatch_gemv(const GemvArgs& a, const Tbl& tbl, bool w_aligned, cudaStream_t s,
                         bool pdl) {
-  const bool nb1 = (a.B == 1);
   const bool aligned = (FMT == GQ_FMT_Q4_0) && (a.rowbytes % 16 == 0) && w_aligned;
-  if (nb1) {
-    return aligned ? launch_gemv<FMT, XT, true, true>(a, tbl, s, pdl)
-                   : launch_gemv<FMT, XT, true, false>(a, tbl, s, pdl);
+  if (a.B == 1) {
+    return aligned ? launch_gemv<FMT, XT, 0, true>(a, tbl, s, pdl)
+                   : launch_gemv<FMT, XT, 0, false>(a, tbl, s, pdl);
   }
-  return aligned ? launch_gemv<FMT, XT, false, true>(a, tbl, s, pdl)
-                 : launch_gemv<FMT, XT, false, false>(a, tbl, s, pdl);
+  if (a.B <= 8) {
+    return aligned ? launch_gemv<FMT, XT, 1, true>(a, tbl, s, pdl)
+                   : launch_gemv<FMT, XT, 1, false>(a, tbl, s, pdl);
+  }
+  return aligned ? launch_gemv<FMT, XT, 2, true>(a, tbl, s, pdl)
+                 : launch_gemv<FMT, XT, 2, false>(a, tbl, s, pdl);
 }
 
 template <int FMT, class Tbl>
@@ -786,7 +837,11 @@ void fill_common(GemvArgs& a, int64_t K, const void* x, int xt, int64_t B, int y
   a.nchunks = static_cast<int>((K + kChunkW - 1) / kChunkW);
   a.skip_first = 0;
   const int terms = (xt == GQ_F32) ? 3 : 1;
-  int win = kXSmemMax / (terms * a.B * kXStride);
+  const int64_t per_chunk = static_cast<int64_t>(terms) * a.B * kXStride;
+  int win = static_cast<int>(kXSmemMax / per_chunk);
+  // batches above 8 keep all of x resident when it fits beside the ring at
+  // one CTA per SM, rather than reloading windows for every row group
+  if (a.B > 8 && per_chunk * a.nchunks <= kXSmemFree) win = a.nchunks;
   if (win < 1) win = 1;
   if (win > a.nchunks) win = a.nchunks;
   a.win = win;
@@ -796,13 +851,13 @@ template <int FMT>
 gq_status gemv_entry(const void* W, int64_t M, int64_t K, const void* x, int xt, int64_t B,
                      void* y, int yt, void* workspace, size_t ws_bytes, unsigned flags,
                      int* dev_status, void* stream, long long budget = kWaitBudget,
-                     int skip_first = 0) {
+                     int skip_first = 0, int64_t max_b = 8) {
   constexpr int kBlkW = Fmt<FMT>::kBlkW;
   if (M < 0 || K < 0 || B < 0) return GQ_ERR_INVALID_ARG;
   if (!valid_act_dtype(xt) || !valid_act_dtype(yt)) return GQ_ERR_DTYPE;
   if (flags & ~GQ_GEMV_PDL) return GQ_ERR_INVALID_ARG;
   if (K % kBlkW) return GQ_ERR_SHAPE;
-  if (B > 8 || M > 0x7FFFFFFFLL || K > (1LL << 24)) return GQ_ERR_SHAPE;
+  if (B > max_b || M > 0x7FFFFFFFLL || K > (1LL << 24)) return GQ_ERR_SHAPE;
   if (M == 0 || B == 0) return GQ_OK;
   if (!y) return GQ_ERR_INVALID_ARG;
   if (misaligned16(y)) return GQ_ERR_ALIGNMENT;
@@ -896,6 +951,16 @@ gq_status gemv_grouped_entry(const gq_gemv_desc* mats, int count, int64_t K, con
 }
 
 }  // namespace
+
+gq_status gemv_batched(int fmt, const void* W, int64_t M, int64_t K, const void* x, int xt,
+                       int64_t B, void* y, int yt, int* dev_status, cudaStream_t stream) {
+  if (fmt == GQ_FMT_Q4_0)
+    return gemv_entry<GQ_FMT_Q4_0>(W, M, K, x, xt, B, y, yt, nullptr, 0, 0u, dev_status, stream,
+                                   kWaitBudget, 0, kWarpMmaMaxB);
+  return gemv_entry<GQ_FMT_KSB>(W, M, K, x, xt, B, y, yt, nullptr, 0, 0u, dev_status, stream,
+                                kWaitBudget, 0, kWarpMmaMaxB);
+}
+
 }  // namespace gq
 
 extern "C" {

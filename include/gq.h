@@ -246,10 +246,15 @@ GQ_API gq_status gq_selftest_gemv_timeout(const void* W, int64_t M, int64_t K, c
  *   X: [B][K] bfloat16 (x_dtype must be GQ_BF16), row-major, 16-byte aligned.
  *   Y: [B][M] of y_dtype (GQ_F32, GQ_F16 or GQ_BF16), row-major.
  *   B: 1..256 (0 launches nothing).
+ * Batches of 1..16 run on the warp-MMA product of gq_gemv_* (each code
+ * decoded once for all columns, two n8 MMA tiles; the workspace is checked
+ * but not used): below about 16 columns a tcgen05 MMA would spend its fixed
+ * cost mostly on empty columns.  Larger batches run on the tcgen05 kernel:
  * Arithmetic: each decoded weight (at most 14 significant bits) is split
  * exactly into two bfloat16 parts, both multiplied by X on the tensor core
  * into one fp32 accumulator, so every product is exact and only the fp32
- * accumulation rounds.
+ * accumulation rounds.  (The warp-MMA path multiplies the exact code - 8 in
+ * bfloat16 and applies the FP16 scale in fp32: also exact products.)
  * Work split: the 128-row tiles x 64-wide k-steps are divided evenly over
  * the SMs (stream-K); a tile shared by two or three SMs is combined through
  * fp32 partial sums, in a fixed order, so results do not depend on

@@ -1,4 +1,5 @@
-"""GPU tensor-core dequant-GEMM against the oracle's fp64 product.
+"""GPU dequant-GEMM against the oracle's fp64 product: batches above 16 run
+on the tcgen05 kernel, batches up to 16 on the warp-MMA product.
 
 Tolerance per output: |Y - Y_ref| <= 1e-4 * sum_k |w_hat||x| plus one unit in
 the last place of the output type.  Weights are quantized by the oracle."""
@@ -109,6 +110,19 @@ def test_gemm_split_shapes(M, K, B):
     # tiles, and the widest batch; checked on rows spanning every tile
     rows = np.unique(np.concatenate([np.arange(0, M, 29), [M - 1]])).astype(np.int64)
     check(Q40, M, K, B, rows=rows)
+
+
+@pytest.mark.parametrize("fmt,M,K,B,ydt", [
+    (Q40, 333, 2080, 9, torch.float32),      # ragged chunk, unaligned rows, odd batch
+    (KSB, 150, 2304, 13, torch.bfloat16),
+    (Q40, 4096, 4096, 16, torch.float32),
+    (KSB, 1000, 4096, 12, torch.float16),
+    (Q40, 17, 8192, 11, torch.float32),
+])
+def test_gemm_warp_mma_batches(fmt, M, K, B, ydt):
+    # batches 9..16 take two n8 tiles of the warp MMA (every code decoded once
+    # for all 16 columns); columns past B are never stored
+    check(fmt, M, K, B, ydt=ydt)
 
 
 def test_gemm_refuses_short_workspace():
