@@ -20,11 +20,12 @@
 //    the CTA that completes it sums every part in CTA order (deterministic)
 //    and resets the tile's count.  CTAs do their (at most two) cut tiles
 //    first.
-//  * warp 0 (producer): streams the tile's packed rows, 512 weights per row
-//    per stage -- one 2-D TMA load of 128 rows x 304 bytes when rows are
-//    whole 16-byte granules, else one 1-D bulk copy per row (no multicast)
-//    -- and the X k-slices (64 x N bf16) with a 2-D TMA load in the
-//    128-byte swizzle;
+//  * warp 0 (W producer): streams the tile's packed rows, 512 weights per
+//    row per stage -- one 2-D TMA load of 128 rows x 304 bytes when rows are
+//    whole 16-byte granules, else one 1-D bulk copy per row (no multicast);
+//  * warp 18 (X producer): the X k-slices (64 x N bf16) with a 2-D TMA load
+//    in the 128-byte swizzle, on their own ring, so that waiting for a free
+//    W stage never delays an activation slice;
 //  * warps 2..9 (dequant, one thread per W row and half k-step): decode
 //    each k-step into the hi and lo bf16 tiles, written straight into the
 //    K-major 128-byte-swizzled UMMA layout, then fence the async proxy;
@@ -65,7 +66,8 @@ constexpr int kATile = kBM * kBK * 2;          // one bf16 tile (hi or lo): 16 K
 constexpr int kStepsPerChunk = kWChunk / kBK;  // 8
 constexpr int kDequantWarps = 8;   // two per scheduler; each thread decodes one block per k-step
 constexpr int kEpiWarps = 8;       // two per TMEM lane quarter, alternate 16-column slices
-constexpr int kThreads = 32 * (2 + kDequantWarps + kEpiWarps);
+constexpr int kXWarp = 2 + kDequantWarps + kEpiWarps;  // the activation producer
+constexpr int kThreads = 32 * (kXWarp + 1);
 
 template <int FMT>
 struct GFmt;
@@ -317,9 +319,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   if (warp == 0) {
-    // ---------------------------------------------------------- producer
-    // Per segment, per k-step: the W chunk (512 weights of the tile's 128
-    // rows) when the step starts one, then the X k-slice.
+    // ------------------------------------------------------- W producer
+    // Per segment, the W chunks (512 weights of the tile's 128 rows) of its
+    // k-steps.  The X k-slices come from their own warp (kXWarp), so that a
+    // wait for a free W stage never holds back an activation load.
     int wseq = 0, g = 0;
     bool ok = true;
     for (int k = 0; k < nseg && ok; ++k) {
@@ -375,16 +378,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ++wseq;
         }
-        const int sx = g % kXStages;
-        if (!mbar_wait(&x_empty[sx], ((g / kXStages) & 1u) ^ 1u, a.budget) || aborted()) {
-          ok = false;
-          break;
-        }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&x_full[sx], L.x_stage);
-          tma_load_2d(gsm + L.x + sx * L.x_stage, &xmap, ks * kBK, 0, &x_full[sx]);
-        }
-        __syncwarp();
       }
     }
     if (!ok && lane == 0) fail();
@@ -392,11 +385,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       for (int c = max(0, wseq - kWStages); c < wseq; ++c)
         if (!mbar_wait(&w_full[c % kWStages], (c / kWStages) & 1u, a.budget)) {
-          report(a.dev_status, GQ_DEV_TIMEOUT);
-          break;
-        }
-      for (int k = max(0, g - kXStages); k < g; ++k)
-        if (!mbar_wait(&x_full[k % kXStages], (k / kXStages) & 1u, a.budget)) {
           report(a.dev_status, GQ_DEV_TIMEOUT);
           break;
         }
@@ -510,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (!ok && lane == 0) fail();
-  } else {
+  } else if (warp < kXWarp) {
     // ---------------------------------------------------------- epilogue
     // TMEM lane quarter = warp % 4: warps 10..17 cover the 128 rows twice,
     // each pair of warps on one quarter splitting the columns
@@ -609,6 +597,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (leader) a.counters[t] = 0;
     }
     if (!ok && lane == 0) fail();
+  } else {
+    // ------------------------------------------------------- X producer
+    // the X k-slice (64 x N bf16, 128-byte swizzle) of every k-step, in the
+    // MMA's order, as far ahead as the X ring allows
+    int g = 0;
+    bool ok = true;
+    for (int k = 0; k < nseg && ok; ++k) {
+      int t, k0, k1;
+      sg.get(k, t, k0, k1);
+      for (int ks = k0; ks < k1; ++ks, ++g) {
+        const int sx = g % kXStages;
+        if (!mbar_wait(&x_empty[sx], ((g / kXStages) & 1u) ^ 1u, a.budget) || aborted()) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&x_full[sx], L.x_stage);
+          tma_load_2d(gsm + L.x + sx * L.x_stage, &xmap, ks * kBK, 0, &x_full[sx]);
+        }
+        __syncwarp();
+      }
+    }
+    if (!ok && lane == 0) fail();
+    // let every issued copy land before shared memory is released
+    if (lane == 0) {
+      for (int k = max(0, g - kXStages); k < g; ++k)
+        if (!mbar_wait(&x_full[k % kXStages], (k / kXStages) & 1u, a.budget)) {
+          report(a.dev_status, GQ_DEV_TIMEOUT);
+          break;
+        }
+    }
   }
 
   // teardown: every MMA has finished before tensor memory is freed
@@ -630,12 +649,21 @@ size_t gemm_smem_bytes(int N, int astages, int xstages) {
 
 // Deepest rings that fit: activations first (their loads wait on the MMA of
 // the slot they refill), then a third decoded-tile stage if room is left.
+// A third decoded-tile stage decouples the dequant warps from the MMA more
+// than X stages beyond four help (X has its own producer), so it is taken
+// first when it fits.
 void choose_stages(int N, int& astages, int& xstages) {
+  const auto fits = [&](int as, int xs) {
+    return gemm_smem_bytes(N, as, xs) <= static_cast<size_t>(kSmemBudget);
+  };
+  for (astages = kAStagesMax; astages > 2; --astages) {
+    for (xstages = kXStagesMax; xstages >= 4 && !fits(astages, xstages); --xstages) {
+    }
+    if (xstages >= 4) return;
+  }
   astages = 2;
   xstages = kXStagesMax;
-  while (xstages > 2 && gemm_smem_bytes(N, astages, xstages) > static_cast<size_t>(kSmemBudget))
-    --xstages;
-  if (gemm_smem_bytes(N, 3, xstages) <= static_cast<size_t>(kSmemBudget)) astages = 3;
+  while (xstages > 2 && !fits(astages, xstages)) --xstages;
 }
 
 // The work split and the workspace it needs: counts of the cut tiles (one
