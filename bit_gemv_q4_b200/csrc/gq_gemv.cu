@@ -952,6 +952,20 @@ gq_status gemv_grouped_entry(const gq_gemv_desc* mats, int count, int64_t K, con
 
 }  // namespace
 
+#if GQ_GEMV_MANY_TU
+// The large-table grouped product, compiled in its own translation unit with
+// the pipeline constants set there (gq_gemv_grouped.cu).
+gq_status gemv_grouped_many(int fmt, const gq_gemv_desc* mats, int count, int64_t K,
+                            const void* x, int xt, int64_t B, int yt, unsigned flags,
+                            int* dev_status, cudaStream_t stream) {
+  if (fmt == GQ_FMT_Q4_0)
+    return gemv_grouped_entry<GQ_FMT_Q4_0>(mats, count, K, x, xt, B, yt, flags, dev_status,
+                                           stream);
+  return gemv_grouped_entry<GQ_FMT_KSB>(mats, count, K, x, xt, B, yt, flags, dev_status, stream);
+}
+
+}  // namespace gq
+#else
 gq_status gemv_batched(int fmt, const void* W, int64_t M, int64_t K, const void* x, int xt,
                        int64_t B, void* y, int yt, int* dev_status, cudaStream_t stream) {
   if (fmt == GQ_FMT_Q4_0)
@@ -960,6 +974,22 @@ gq_status gemv_batched(int fmt, const void* W, int64_t M, int64_t K, const void*
   return gemv_entry<GQ_FMT_KSB>(W, M, K, x, xt, B, y, yt, nullptr, 0, 0u, dev_status, stream,
                                 kWaitBudget, 0, kWarpMmaMaxB);
 }
+
+// Row groups of a grouped call's valid descriptors (validation happens in
+// the entry point that is then chosen).
+int64_t grouped_groups(const gq_gemv_desc* mats, int count) {
+  int64_t g = 0;
+  for (int i = 0; mats && i < count; ++i)
+    if (mats[i].M > 0) g += (mats[i].M + kRows - 1) / kRows;
+  return g;
+}
+
+// Grouped calls with at least this many row groups per SM stream on the
+// large-table configuration (four small CTAs per SM, gq_gemv_grouped.cu):
+// with that much work per SM, more independent pipelines per SM beat fewer
+// wide ones, while a single matrix or a short table keeps this file's
+// configuration (wide CTAs whose early exit lets the next launch start).
+constexpr int64_t kManyGroupsPerSm = 8;
 
 }  // namespace gq
 
@@ -990,6 +1020,9 @@ GQ_API gq_status gq_gemv_ksb(const void* W, int64_t M, int64_t K, const void* x,
 GQ_API gq_status gq_gemv_q4_0_grouped(const gq_gemv_desc* mats, int count, int64_t K,
                                       const void* x, int x_dtype, int64_t B, int y_dtype,
                                       unsigned flags, int* dev_status, void* stream) {
+  if (count > 0 && gq::grouped_groups(mats, count) >= gq::kManyGroupsPerSm * gq::sm_count())
+    return gq::gemv_grouped_many(GQ_FMT_Q4_0, mats, count, K, x, x_dtype, B, y_dtype, flags,
+                                 dev_status, gq::as_stream(stream));
   return gq::gemv_grouped_entry<GQ_FMT_Q4_0>(mats, count, K, x, x_dtype, B, y_dtype, flags,
                                              dev_status, stream);
 }
@@ -997,6 +1030,9 @@ GQ_API gq_status gq_gemv_q4_0_grouped(const gq_gemv_desc* mats, int count, int64
 GQ_API gq_status gq_gemv_ksb_grouped(const gq_gemv_desc* mats, int count, int64_t K,
                                      const void* x, int x_dtype, int64_t B, int y_dtype,
                                      unsigned flags, int* dev_status, void* stream) {
+  if (count > 0 && gq::grouped_groups(mats, count) >= gq::kManyGroupsPerSm * gq::sm_count())
+    return gq::gemv_grouped_many(GQ_FMT_KSB, mats, count, K, x, x_dtype, B, y_dtype, flags,
+                                 dev_status, gq::as_stream(stream));
   return gq::gemv_grouped_entry<GQ_FMT_KSB>(mats, count, K, x, x_dtype, B, y_dtype, flags,
                                             dev_status, stream);
 }
@@ -1032,3 +1068,4 @@ GQ_API gq_status gq_selftest_gemv_timeout(const void* W, int64_t M, int64_t K, c
 }
 
 }  // extern "C"
+#endif  // GQ_GEMV_MANY_TU

@@ -20,4 +20,13 @@ constexpr int64_t kWarpMmaMaxB = 16;
 gq_status gemv_batched(int fmt, const void* W, int64_t M, int64_t K, const void* x, int xt,
                        int64_t B, void* y, int yt, int* dev_status, cudaStream_t stream);
 
+// gq_gemv_*_grouped on the large-table configuration (gq_gemv_grouped.cu:
+// four small CTAs per SM, 1024-weight chunks), for tables with many row
+// groups per SM.  Arguments, validation and status as for the grouped entry
+// points; results differ from the single-matrix product only in the order
+// of fp32 additions.
+gq_status gemv_grouped_many(int fmt, const gq_gemv_desc* mats, int count, int64_t K,
+                            const void* x, int xt, int64_t B, int yt, unsigned flags,
+                            int* dev_status, cudaStream_t stream);
+
 }  // namespace gq

@@ -191,7 +191,10 @@ GQ_API gq_status gq_gemv_ksb(const void* W, int64_t M, int64_t K,
  * The pages stream one matrix at a time; this entry point has no counterpart
  * on them.  One launch covers up to 256 matrices: its CTAs load x once and
  * stream the 16-row groups of all of them back to back, so there is no
- * launch gap and no repeated activation load between matrices.
+ * launch gap and no repeated activation load between matrices.  Tables with
+ * fewer than 8 row groups per SM give each output bit for bit what
+ * gq_gemv_* gives; larger ones run a pipeline shaped for long streams whose
+ * results differ from it only in the order of fp32 additions.
  *   mats:  count host descriptors {W, M, y} (read during the call only).  W as
  *          for gq_gemv_*, 16-byte aligned; y: [B][M] of y_dtype, 16-byte
  *          aligned.  M == 0 entries are skipped (W and y may then be NULL).

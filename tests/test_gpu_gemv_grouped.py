@@ -1,8 +1,9 @@
 """Grouped GEMV (gq_gemv_*_grouped): several matrices sharing K and x in one
 launch.  Every output is compared with the oracle's fp64 product (tolerance as
-in test_gpu_gemv.py) and with the single-matrix entry point, which computes
-each row with the same arithmetic in the same order, so the two agree bit for
-bit."""
+in test_gpu_gemv.py).  Tables with fewer than 8 row groups per SM run on the
+single-matrix configuration and agree with the single-matrix entry point bit
+for bit; larger tables run on the large-table configuration (four small CTAs
+per SM), whose sums differ only in the order of fp32 additions."""
 import numpy as np
 import pytest
 import torch
@@ -82,18 +83,43 @@ def test_grouped_more_matrices_than_one_launch():
 
 
 def test_grouped_model_layer_shapes():
-    # one decoder layer of the whole-model stream: 4 x 4096^2 and 3 x 11008x4096,
-    # one x; checked against the single-matrix calls
+    # one decoder layer of the whole-model stream (4 x 4096^2 and 3 x
+    # 11008x4096, 3088 row groups: the large-table configuration), one x;
+    # checked against the oracle on rows spanning every 16-row group boundary
     K = 4096
     Ms = [4096, 4096, 4096, 4096, 11008, 11008, 4096]
-    rng_seeds = 30000
-    Wd, ys = [], []
+    assert sum((M + 15) // 16 for M in Ms) >= 8 * torch.cuda.get_device_properties(0).multi_processor_count
     x = synth.activations(1, K, seed=9, dtype=torch.float16).cuda()
+    Wd = []
     for i, M in enumerate(Ms):
-        w = synth.gaussian_weights(M, K, seed=rng_seeds + i, device="cuda")
-        W = gq.gq_quantize_q4_0(w.view(-1))
-        Wd.append(W)
-        ys.append(_single(Q40, W, M, K, x, torch.float16))
+        w = synth.gaussian_weights(M, K, seed=30000 + i, device="cuda")
+        Wd.append(gq.gq_quantize_q4_0(w.view(-1)))
     outs = _grouped(Q40, Wd, Ms, K, x, torch.float16, flags=gq.GQ_GEMV_PDL)
-    for y, ys_ in zip(outs, ys):
-        assert torch.equal(y.view(torch.int16), ys_.view(torch.int16))
+    xo, xt = x_for_oracle(x)
+    for W, M, y in zip(Wd, Ms, outs):
+        rows = np.unique(np.concatenate([np.arange(0, M, 53), np.arange(15, M, 211), [M - 1]]))
+        Yr, bound = oracle.gemm_rows(Q40, W.cpu().numpy(), M, K, xo, rows.astype(np.int64), xt)
+        assert_product_close(y[:, torch.from_numpy(rows).cuda()], Yr, bound)
+
+
+@pytest.mark.parametrize("fmt", [Q40, KSB])
+def test_grouped_large_table_ragged(fmt):
+    # 1300 matrices of 1..40 rows (about 2000 row groups: the large-table
+    # configuration, in six launches of up to 256 matrices) against the oracle
+    K = 512 if fmt == Q40 else 768
+    rng = np.random.default_rng(3)
+    Ms = [int(m) for m in rng.integers(1, 41, size=1300)]
+    assert sum((M + 15) // 16 for M in Ms) >= 8 * torch.cuda.get_device_properties(0).multi_processor_count
+    w = synth.gaussian_weights(sum(Ms), K, seed=17).numpy()
+    qs, r0 = [], 0
+    for M in Ms:
+        q, _ = oracle.quantize(fmt, w[r0:r0 + M].ravel())
+        qs.append(q)
+        r0 += M
+    Wd = [torch.from_numpy(q).cuda() for q in qs]
+    x = synth.activations(2, K, seed=4, dtype=torch.bfloat16).cuda()
+    outs = _grouped(fmt, Wd, Ms, K, x, torch.float32, flags=gq.GQ_GEMV_PDL)
+    xo, xt = x_for_oracle(x)
+    for q, M, y in zip(qs, Ms, outs):
+        Y, bound = oracle.gemm(fmt, q, M, K, xo, xt)
+        assert_product_close(y, Y, bound)
