@@ -775,7 +775,7 @@ gq_status gemm_entry(const void* W, int64_t M, int64_t K, const void* X, int xt,
 
   choose_stages(N, a.astages, a.xstages);
   const size_t smem = gemm_smem_bytes(N, a.astages, a.xstages);
-  static int configured_dev = -1;
+  thread_local int configured_dev = -1;  // per host thread (concurrent callers)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
   if (configured_dev != dev) {

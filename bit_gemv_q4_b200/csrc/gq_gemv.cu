@@ -764,10 +764,12 @@ gq_status launch_gemv(const GemvArgs& a, const Tbl& tbl, cudaStream_t stream, bo
   constexpr int kTerms = (XT == XT_F32) ? 3 : 1;
   auto kern = gemv_kernel<FMT, XT, NT, ALIGNED, Tbl>;
   const size_t smem = gemv_smem_bytes(a.B, kTerms, a.win);
-  static int configured_dev = -1;
-  static size_t configured_smem = 0;
-  static size_t occ_smem = 0;
-  static int occupancy = 1;
+  // per host thread, so that concurrent callers (possibly on other devices)
+  // never see each other's half-updated state
+  thread_local int configured_dev = -1;
+  thread_local size_t configured_smem = 0;
+  thread_local size_t occ_smem = 0;
+  thread_local int occupancy = 1;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
   if (configured_dev != dev || smem > configured_smem) {

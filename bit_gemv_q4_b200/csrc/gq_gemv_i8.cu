@@ -50,6 +50,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "gq.h"
 #include "gq_device.cuh"
 #include "gq_gemv_i8.h"
@@ -610,7 +612,7 @@ gq_status i8_gemv(const void* W, int64_t M, int64_t K, const void* x, void* y, i
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return GQ_ERR_CUDA;
 
-  static int configured_dev = -1;
+  thread_local int configured_dev = -1;  // per host thread (concurrent callers)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
   if (configured_dev != dev) {
@@ -643,15 +645,15 @@ namespace gq {
 // Address of the static scratch on the current device, looked up once per
 // device (the first call on a device should come before any stream capture).
 static gq_status noalloc_scratch(uint8_t** out) {
-  static void* addr[64] = {nullptr};
+  static std::atomic<void*> addr[64];  // zero-initialized; same value from every thread
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GQ_ERR_CUDA;
-  if (!addr[dev]) {
-    void* p = nullptr;
+  void* p = addr[dev].load(std::memory_order_relaxed);
+  if (!p) {
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GQ_ERR_CUDA;
-    addr[dev] = p;
+    addr[dev].store(p, std::memory_order_relaxed);
   }
-  *out = static_cast<uint8_t*>(addr[dev]);
+  *out = static_cast<uint8_t*>(p);
   return GQ_OK;
 }
 

@@ -123,3 +123,40 @@ def test_misaligned_rows_large_k():
     y = run_gemv(KSB, q, M, K, x, torch.float32)
     Y, bound = oracle.gemm(KSB, q, M, K, *x_for_oracle(x))
     assert_product_close(y, Y, bound)
+
+
+def test_concurrent_host_threads():
+    # several host threads launch products of different shapes (different
+    # shared-memory sizes and kernel configurations) on their own streams at
+    # once; every result equals the same call made alone
+    import threading
+    cases = [(Q40, 4096, 4096, 1), (KSB, 300, 11008, 1), (Q40, 1000, 2048, 8), (KSB, 129, 4352, 3)]
+    data = []
+    for fmt, M, K, B in cases:
+        q = torch.from_numpy(packed(fmt, M, K)).cuda()
+        x = synth.activations(B, K, seed=M + B, dtype=torch.float16).cuda()
+        f = gq.gq_gemv_q4_0 if fmt == Q40 else gq.gq_gemv_ksb
+        ref = f(q, M, K, x, y_dtype=torch.float32)
+        data.append((f, q, M, K, x, ref))
+    torch.cuda.synchronize()
+    errors = []
+
+    def worker(i):
+        try:
+            f, q, M, K, x, ref = data[i % len(data)]
+            s = torch.cuda.Stream()
+            with torch.cuda.stream(s):
+                for _ in range(20):
+                    y = f(q, M, K, x, y_dtype=torch.float32, stream=s)
+            s.synchronize()
+            if not torch.equal(y, ref):
+                errors.append(i)
+        except Exception as e:  # reported below
+            errors.append(repr(e))
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(8)]
+    for th in threads:
+        th.start()
+    for th in threads:
+        th.join()
+    assert not errors, errors
