@@ -364,7 +364,20 @@ __device__ __forceinline__ void q40_chunk(float* acc, uint32_t row0, uint32_t ro
 // A consumer warp's kSubPerWarp sub-blocks of one super-block of the stage.
 // s~_j = S * q_j is applied as q_j per sub-block and S once at the end.  All
 // loads are issued before the first decode.
-template <int XT, int NT>
+// MIS: offset mod 4 of the super-block's code and sub-scale words when rows
+// are 16-byte aligned (then fixed per warp: 138-byte super-blocks alternate
+// between 0 and 2 mod 4 and chunks start on multiples of 8 bytes); -1 when
+// it is known only at run time.
+template <int MIS>
+__device__ __forceinline__ uint32_t ld32_w(uint32_t off) {
+  if constexpr (MIS < 0) {
+    return ld32_even(off);
+  } else {
+    return ld32_at<MIS>(off);
+  }
+}
+
+template <int XT, int NT, int MIS>
 __device__ __forceinline__ void ksb_chunk(float* acc, uint32_t row0, uint32_t row1, uint32_t xw,
                                           uint32_t term_stride, uint32_t xt1, int w, int t) {
   constexpr bool kOne = (NT == 0);
@@ -377,11 +390,11 @@ __device__ __forceinline__ void ksb_chunk(float* acc, uint32_t row0, uint32_t ro
   const float Sa = half_bits_to_float(ld16(sa));
   const float Sb = kOne ? Sa : half_bits_to_float(ld16(b));
   uint32_t qja[2], qjb[2];
-  qja[0] = ld32_even(sa + 2 + j0);
-  qjb[0] = kOne ? qja[0] : ld32_even(b + 2 + j0);
+  qja[0] = ld32_w<MIS>(sa + 2 + j0);
+  qjb[0] = kOne ? qja[0] : ld32_w<MIS>(b + 2 + j0);
   if constexpr (kSubPerWarp > 4) {
-    qja[1] = ld32_even(sa + 6 + j0);
-    qjb[1] = kOne ? qja[1] : ld32_even(b + 6 + j0);
+    qja[1] = ld32_w<MIS>(sa + 6 + j0);
+    qjb[1] = kOne ? qja[1] : ld32_w<MIS>(b + 6 + j0);
   }
   float sacc[acc_len(NT)];
 #pragma unroll
@@ -392,8 +405,8 @@ __device__ __forceinline__ void ksb_chunk(float* acc, uint32_t row0, uint32_t ro
     uint32_t na[kBatch], nb[kBatch];
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
-      na[j] = ld32_even(a + 10 + 16 * (j0 + h + j) + 4 * t);
-      nb[j] = ld32_even(b + 10 + 16 * (j0 + h + j) + 4 * t);
+      na[j] = ld32_w<MIS>(a + 10 + 16 * (j0 + h + j) + 4 * t);
+      nb[j] = ld32_w<MIS>(b + 10 + 16 * (j0 + h + j) + 4 * t);
     }
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
@@ -684,9 +697,18 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
                                    xw, term_stride, xt1, cw, t, nvalid);
         }
       } else {
-        if (whole || tail_valid)
-          ksb_chunk<XT, NT>(acc, stg + r * kPitch + off0, stg + (r + 8) * kPitch + off1, xw,
-                            term_stride, xt1, cw, t);
+        if (whole || tail_valid) {
+          const uint32_t p0 = stg + r * kPitch + off0, p1 = stg + (r + 8) * kPitch + off1;
+          if constexpr (ALIGNED) {
+            // this warp's super-block: even ones put their words at 2 mod 4
+            if (((cw * kSubPerWarp) >> 3) & 1)
+              ksb_chunk<XT, NT, 0>(acc, p0, p1, xw, term_stride, xt1, cw, t);
+            else
+              ksb_chunk<XT, NT, 2>(acc, p0, p1, xw, term_stride, xt1, cw, t);
+          } else {
+            ksb_chunk<XT, NT, -1>(acc, p0, p1, xw, term_stride, xt1, cw, t);
+          }
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
@@ -801,7 +823,9 @@ gq_status launch_gemv(const GemvArgs& a, const Tbl& tbl, cudaStream_t stream, bo
 template <int FMT, int XT, class Tbl>
 gq_status dispatch_gemv(const GemvArgs& a, const Tbl& tbl, bool w_aligned, cudaStream_t s,
                         bool pdl) {
-  const bool aligned = (FMT == GQ_FMT_Q4_0) && (a.rowbytes % 16 == 0) && w_aligned;
+  // Q4_0 rows of whole granules keep every chunk on a 16-byte boundary; ksb
+  // rows of whole granules fix each warp's word alignment (ksb_chunk)
+  const bool aligned = (a.rowbytes % 16 == 0) && w_aligned;
   if (a.B == 1) {
     return aligned ? launch_gemv<FMT, XT, 0, true>(a, tbl, s, pdl)
                    : launch_gemv<FMT, XT, 0, false>(a, tbl, s, pdl);
