@@ -194,6 +194,46 @@ def test_outlier_demo_page_reference_rule():
     assert rec[31] == 10.0 and np.all(rec[:31] == 0.0)
 
 
+@pytest.mark.parametrize("first_sign", [1.0, -1.0])
+def test_reference_rule_hand_worked_block(first_sign):
+    # a block worked by hand under section 4.4's printed rule, with values
+    # whose products with 1/d are exact in fp32: the max magnitude 4 occurs
+    # twice with opposite signs and the first one sets d = max / -8;
+    # codes are min(15, trunc(x / d + 8.5)) -- truncation, not rounding
+    s = first_sign
+    x = np.zeros(32, np.float32)
+    x[5], x[9] = 4.0 * s, -4.0 * s        # tie in magnitude: position 5 wins
+    x[1], x[2], x[3], x[4] = 1.0 * s, -1.0 * s, 0.75 * s, 0.5 * s
+    x[6], x[7] = 0.25 * s, -0.25 * s
+    q, flags = oracle.quantize_q4_0(x, rule=oracle.RULE_LLAMA)
+    assert flags == 0
+    d = float(oracle.f16_bits_to_f32([_u16(q, 0)])[0])
+    assert d == -0.5 * s                  # 4s / -8
+    codes = np.concatenate([q[2:] & 0xF, q[2:] >> 4])
+    # x / d = -2x/s: 4s -> -8 + 8.5 = 0.5 -> 0; -4s -> 16.5 -> min(15, 16) = 15;
+    # s -> 6.5 -> 6; -s -> 10.5 -> 10; 0.75s -> 7.0 -> 7; 0.5s -> 7.5 -> 7;
+    # 0.25s -> 8.0 -> 8; -0.25s -> 9.0 -> 9; 0 -> 8.5 -> 8
+    want = {5: 0, 9: 15, 1: 6, 2: 10, 3: 7, 4: 7, 6: 8, 7: 9}
+    for i in range(32):
+        assert codes[i] == want.get(i, 8), (i, codes[i])
+
+
+def test_reference_rule_zero_and_truncation_edges():
+    # a zero block: d = 0 / -8 = -0, the inverse scale is taken as 0, every
+    # code is trunc(8.5) = 8 and the stored scale is FP16 -0
+    q, _ = oracle.quantize_q4_0(np.zeros(32, np.float32), rule=oracle.RULE_LLAMA)
+    assert _u16(q, 0) == 0x8000 and np.all(q[2:] == 0x88)
+    # max 8 -> d = -1, id = -1: x = 0.4 gives 8.1 -> 8, x = -0.6 gives 9.1 -> 9
+    # (round-to-nearest would give 8 and 9 as well; x = -0.4 gives 8.9 -> 8,
+    # where rounding would give 9)
+    x = np.zeros(32, np.float32)
+    x[0], x[1], x[2], x[3] = 8.0, 0.4, -0.6, -0.4
+    q, _ = oracle.quantize_q4_0(x, rule=oracle.RULE_LLAMA)
+    codes = np.concatenate([q[2:] & 0xF, q[2:] >> 4])
+    assert _u16(q, 0) == 0xBC00           # FP16 -1.0
+    assert codes[0] == 0 and codes[1] == 8 and codes[2] == 9 and codes[3] == 8
+
+
 def test_outlier_demo_build_rule():
     # the build's rule d = FP16(absmax/7): the outlier still takes the top code
     # and every small value collapses to zero (the failure mode the page shows)
