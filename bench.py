@@ -41,7 +41,7 @@ FALLBACK_HBM_GBS = 6650.0
 GEMV_TRAFFIC = {
     "bytes": 25407744,
     "sources": {
-        "bit_gemv_q4_b200/csrc/gq_gemv.cu": "9d0b62d3394264203c880ff2b7603583e2c4075182916261cf4ac1768764548e",
+        "bit_gemv_q4_b200/csrc/gq_gemv.cu": "2097710892fc724426aeafb75a26e0e3488edc2a224265dbdbaa265152e66880",
         "bit_gemv_q4_b200/csrc/gq_device.cuh": "c88e136b756c0355212db717041e37b38523df1a913fe4fa63cd047c2a12e5f4",
     },
 }
