@@ -285,6 +285,16 @@ def run_ours(args, rank, ws, local):
     nopdl_gbs = wbytes_step * max(20, args.steps // 10) / (ms_nopdl / 1e3) / 1e9
     del g_nopdl
 
+    # practical ceiling: the same weight copies read once each by a plain
+    # streaming-read kernel (gq_stream_read), one launch per matrix, same graph
+    sink = torch.zeros(1, dtype=torch.int32, device=dev)
+    g_read = capture(lambda: [gq.gq_stream_read(s["W"][c], sink) for s in sets
+                              for c in range(copies)])
+    read_steps = max(20, args.steps // 10)
+    ms_read = time_graph(g_read, read_steps, args.warmup, ws)
+    read_gbs = wbytes_step * read_steps / (ms_read / 1e3) / 1e9
+    del g_read
+
     # end to end through the public API with host buffers: each step copies
     # the four activation vectors from pinned host memory, runs the step's
     # GEMVs and reads the four results back into pinned host memory
@@ -345,6 +355,10 @@ def run_ours(args, rank, ws, local):
                      "kernel": "gemv_kernel (all four cases)"},
         "cases": cases,
         "no_pdl_gbs": round(nopdl_gbs, 1),
+        "read_ceiling": {"gbs": round(read_gbs, 1), "frac_of_peak": round(read_gbs / peak, 4),
+                         "value_frac_of_ceiling": round(gbs / ws / read_gbs, 4),
+                         "what": "the same weight copies, one plain streaming-read launch "
+                                 "(gq_stream_read) per matrix, same CUDA graph"},
         "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "mode": e2e_mode},
         "gpu_launches": launches,
@@ -491,6 +505,22 @@ def run_suite(path):
               "frac_of_peak": round(nb / (ms * 1e-3) / 1e9 / peak, 4),
               "gflops": round(2 * M * K * B / (ms * 1e-3) / 1e9, 1)})
         del Wc
+
+    # --- read ceiling of one launch: the same rotated copies of each headline
+    # matrix read once by a plain streaming-read kernel, graph of launches
+    sink = torch.zeros(1, dtype=torch.int32, device=dev)
+    for fmt, M, K in CASES:
+        nb = packed_bytes(fmt, M, K)
+        copies = max(4, int(512e6 // nb))
+        buf = torch.empty((copies, nb), dtype=torch.uint8, device=dev)
+        buf.fill_(7)
+        ms = _graph_ms_per_launch(lambda: [gq.gq_stream_read(buf[i], sink) for i in range(copies)],
+                                  copies, 20)
+        emit({"row": "read_ceiling", "workload": f"plain streaming read of one {fmt} {M}x{K} "
+              "matrix per launch", "bytes": nb, "us": round(ms * 1e3, 3),
+              "gbs": round(nb / (ms * 1e-3) / 1e9, 1),
+              "frac_of_peak": round(nb / (ms * 1e-3) / 1e9 / peak, 4)})
+        del buf
 
     # --- whole-model weight stream: 32 layers x (4 x 4096^2 + 3 x 11008x4096)
     for fmt in ("q4_0", "ksb"):

@@ -34,7 +34,7 @@ EXPORTS = (
     "gq_gemv_workspace_bytes", "gq_gemv_q4_0", "gq_gemv_ksb",
     "gq_gemv_q4_0_grouped", "gq_gemv_ksb_grouped",
     "gq_gemm_workspace_bytes", "gq_gemm_q4_0", "gq_gemm_ksb",
-    "gq_selftest_gemv_timeout", "gq_gemv_q4_0_noalloc",
+    "gq_selftest_gemv_timeout", "gq_gemv_q4_0_noalloc", "gq_stream_read",
 )
 
 _DTYPE_CODE = {torch.float32: GQ_F32, torch.float16: GQ_F16, torch.bfloat16: GQ_BF16}
@@ -92,6 +92,8 @@ def _load() -> ctypes.CDLL:
     L.gq_gemv_q4_0_noalloc.restype = c_int
     L.gq_selftest_gemv_timeout.argtypes = [vp, i64, i64, vp, vp, vp, vp]
     L.gq_selftest_gemv_timeout.restype = c_int
+    L.gq_stream_read.argtypes = [vp, ctypes.c_size_t, vp, vp]
+    L.gq_stream_read.restype = c_int
     return L
 
 
@@ -360,3 +362,15 @@ def gq_selftest_gemv_timeout(W: torch.Tensor, M: int, K: int, x: torch.Tensor, y
     _check(lib.gq_selftest_gemv_timeout(_ptr(W), int(M), int(K), _ptr(x), _ptr(y),
                                         _ptr(dev_status), _stream(stream)),
            "gq_selftest_gemv_timeout")
+
+
+def gq_stream_read(buf: torch.Tensor, sink: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """Read every byte of `buf` once on the GPU and XOR its 32-bit words into
+    `sink` (an int32 tensor of one element, zeroed here when not given): the
+    practical read ceiling of one launch of that size."""
+    if sink is None:
+        sink = torch.zeros(1, dtype=torch.int32, device=buf.device)
+    nbytes = buf.numel() * buf.element_size()
+    _check(lib.gq_stream_read(_ptr(buf), nbytes, _ptr(sink), _stream(stream)), "gq_stream_read")
+    return sink

@@ -242,6 +242,18 @@ GQ_API gq_status gq_gemv_q4_0_noalloc(const void* W, int64_t M, int64_t K, const
 GQ_API gq_status gq_selftest_gemv_timeout(const void* W, int64_t M, int64_t K, const void* x,
                                           void* y, int* dev_status, void* stream);
 
+/* Calibration (no counterpart on the pages): reads `bytes` bytes at p once
+ * with 16-byte streaming loads and XORs every little-endian 32-bit word of
+ * them into *sink (device memory; the caller zeroes it first, the fold is
+ * applied with atomics).  One launch of this is the practical ceiling for a
+ * kernel that reads that many bytes once, launch and drain included: the
+ * reference the GEMV's streamed-weight rate is compared with beside the
+ * long-copy peak.
+ *   p: device pointer, 16-byte aligned (GQ_ERR_ALIGNMENT); bytes % 16 == 0
+ *   (GQ_ERR_SHAPE); sink: 4-byte aligned device word.  bytes == 0 launches
+ *   nothing.  Asynchronous on `stream`. */
+GQ_API gq_status gq_stream_read(const void* p, size_t bytes, uint32_t* sink, void* stream);
+
 /* Dequantize-fused batched product for batches that make a dense
  * contraction: Y = W_hat * X^T on the tcgen05 tensor cores (the matrix
  * multiply that consumes decoded blocks, Q4_0 chapter 4.3).
