@@ -39,10 +39,10 @@ FALLBACK_HBM_GBS = 6650.0
 # one ncu capture (profiles/gemv_q4_0_4096x11008.md).  Reported only while the
 # GEMV sources hash to what was profiled; any change to the kernel makes it null.
 GEMV_TRAFFIC = {
-    "bytes": 25407744,
+    "bytes": 25406976,
     "sources": {
         "bit_gemv_q4_b200/csrc/gq_gemv.cu": "2097710892fc724426aeafb75a26e0e3488edc2a224265dbdbaa265152e66880",
-        "bit_gemv_q4_b200/csrc/gq_device.cuh": "c88e136b756c0355212db717041e37b38523df1a913fe4fa63cd047c2a12e5f4",
+        "bit_gemv_q4_b200/csrc/gq_device.cuh": "8eec6074ffd6e2337bf1ea2999f16285b22b3bca681a3cbf9c4acd0b821173c2",
     },
 }
 
@@ -575,8 +575,12 @@ def run_suite(path):
         for B in (16, 64, 256):
             X = synth.activations(B, K, seed=12, dtype=torch.bfloat16, device=dev)
             Y = torch.empty((B, M), dtype=torch.float32, device=dev)
-            ms = _graph_ms_per_launch(lambda: [f(Wc[i], M, K, X, out=Y) for i in range(copies)],
-                                      copies, 10)
+            # one zeroed workspace for every call: a call leaves it ready for the next
+            code = gq.GQ_FMT_Q4_0 if fmt == "q4_0" else gq.GQ_FMT_KSB
+            wsp = torch.zeros(max(gq.gq_gemm_workspace_bytes(code, M, K, B), 1), dtype=torch.uint8,
+                              device=dev)
+            ms = _graph_ms_per_launch(
+                lambda: [f(Wc[i], M, K, X, out=Y, workspace=wsp) for i in range(copies)], copies, 10)
             tf = 2.0 * M * K * B / (ms * 1e-3) / 1e12
             emit({"row": "gemm", "workload": f"W {M}x{K} x X bf16 [{B},{K}], Y fp32",
                   "format": fmt, "B": B, "us": round(ms * 1e3, 2), "tflops": round(tf, 1),
