@@ -349,6 +349,7 @@ def run_ours(args, rank, ws, local):
             "parallelism": "replicas" if ws > 1 else "single GPU",
         },
         "frac_of_peak": round(gbs / ws / peak, 4),
+        "frac_of_nominal_8tbs": round(gbs / ws / 8000.0, 4),
         "roofline": {"bound": "hbm", "achieved": round(per_gpu_algo_gbs, 1), "peak": peak,
                      "peak_source": f"{peak_src} hbm_gbs", "unit": "GB/s",
                      "frac": round(per_gpu_algo_gbs / peak, 4), "traffic": gemv_traffic(),
