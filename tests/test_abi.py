@@ -211,3 +211,13 @@ def test_gemv_workspace_sizes_and_checks():
     # too small, then misaligned: both refused before any launch
     assert f(*args, A, need - 1, 0, None, None) == 9
     assert f(*args, A + 16, need, 0, None, None) == ALIGN
+
+
+def test_stream_read_validation():
+    f = gq.lib.gq_stream_read
+    assert f(A, 64, None, None) == INVALID  # no sink
+    assert f(None, 64, A, None) == INVALID  # bytes but no buffer
+    assert f(A, 40, A, None) == SHAPE  # not whole 16-byte granules
+    assert f(A + 8, 64, A, None) == ALIGN  # buffer off a 16-byte boundary
+    assert f(A, 64, A + 2, None) == ALIGN  # sink off a 4-byte boundary
+    assert f(None, 0, A, None) == GQ_OK  # nothing to read: no launch
