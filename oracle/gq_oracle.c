@@ -154,25 +154,42 @@ static int quant_block_absmax7(const float* x, uint8_t* out) {
     return flags;
 }
 
-/* The page's reference quantizer ([Q40] 4.4): the signed value of largest
- * magnitude sets d = max / -8; codes are min(15, trunc(x * (1/d) + 8.5)). */
+/* The element of largest magnitude, with its sign; among equal magnitudes
+ * the one seen first ([Q40] 4.4: the scan keeps its candidate unless a later
+ * value is strictly larger in magnitude).  A block of zeros gives +0. */
+static float signed_absmax_first(const float* x, int n) {
+    float best = 0.0f;
+    for (int i = 0; i < n; ++i)
+        if (fabsf(x[i]) > fabsf(best)) best = x[i];
+    return best;
+}
+
+/* One 4-bit code under the page's reference rule ([Q40] 4.4): the value is
+ * multiplied by the inverse scale, shifted by 8.5 and truncated toward zero,
+ * each operation rounded to fp32; the result is capped at 15.  Below zero
+ * (only reachable through rounding) the code is 0. */
+static int code_ref_rule(float x, float inv_d) {
+    float shifted = x * inv_d;
+    shifted = shifted + 8.5f;
+    if (!(shifted >= 0.0f) || !(shifted < 1e9f)) return 0;
+    int c = (int)shifted;
+    return c > 15 ? 15 : c;
+}
+
+/* Block quantizer of the page's reference rule ([Q40] 4.4, demonstrated on
+ * the outlier block of 4.5): the scale is d = vmax / -8 for the signed value
+ * vmax of largest magnitude, so vmax itself lands on code 0; the inverse
+ * scale is 1/d, or 0 for a zero scale (every code then 8). */
 static int quant_block_llama(const float* x, uint8_t* out) {
     int flags = ORC_OK;
-    float amax = 0.0f, vmax = 0.0f;
-    for (int i = 0; i < Q40_BLOCK; ++i) {
+    for (int i = 0; i < Q40_BLOCK; ++i)
         if (!isfinite(x[i])) flags |= ORC_NONFINITE;
-        if (amax < fabsf(x[i])) { amax = fabsf(x[i]); vmax = x[i]; }
-    }
-    float d = vmax / -8.0f;
-    float id = (d != 0.0f) ? 1.0f / d : 0.0f;
-    uint16_t d16 = orc_f32_to_f16(d);
+    const float d = signed_absmax_first(x, Q40_BLOCK) / -8.0f;
+    const float inv_d = (d == 0.0f) ? 0.0f : 1.0f / d;
+    const uint16_t d16 = orc_f32_to_f16(d);
     if ((d16 & 0x7FFFu) == 0x7C00u) flags |= ORC_RANGE;
     int c[32];
-    for (int i = 0; i < Q40_BLOCK; ++i) {
-        float t = x[i] * id + 8.5f;
-        int v = (t >= 0.0f && t < 1e9f) ? (int)t : 0;
-        c[i] = v < 15 ? v : 15;
-    }
+    for (int i = 0; i < Q40_BLOCK; ++i) c[i] = code_ref_rule(x[i], inv_d);
     put_u16le(out, d16);
     pack_32(c, out + 2);
     return flags;

@@ -82,24 +82,50 @@ def test_grouped_more_matrices_than_one_launch():
         assert_product_close(y, Y, bound)
 
 
-def test_grouped_model_layer_shapes():
-    # one decoder layer of the whole-model stream (4 x 4096^2 and 3 x
-    # 11008x4096, 3088 row groups: the large-table configuration), one x;
-    # checked against the oracle on rows spanning every 16-row group boundary
-    K = 4096
-    Ms = [4096, 4096, 4096, 4096, 11008, 11008, 4096]
+def _every_group_rows(M):
+    """One row in every 16-row group (its position inside the group varies)
+    plus the last row."""
+    g = np.arange((M + 15) // 16)
+    rows = np.minimum(16 * g + (5 * g) % 16, M - 1)
+    return np.unique(np.concatenate([rows, [M - 1]])).astype(np.int64)
+
+
+def _large_table_case(fmt, Ms, K, seed, ydt=torch.float16):
+    """Oracle-quantized matrices in one grouped call that takes the
+    large-table configuration; each output checked on one row of every 16-row
+    group against the oracle's fp64 product."""
     assert sum((M + 15) // 16 for M in Ms) >= 8 * torch.cuda.get_device_properties(0).multi_processor_count
-    x = synth.activations(1, K, seed=9, dtype=torch.float16).cuda()
-    Wd = []
-    for i, M in enumerate(Ms):
-        w = synth.gaussian_weights(M, K, seed=30000 + i, device="cuda")
-        Wd.append(gq.gq_quantize_q4_0(w.view(-1)))
-    outs = _grouped(Q40, Wd, Ms, K, x, torch.float16, flags=gq.GQ_GEMV_PDL)
+    x = synth.activations(1, K, seed=seed, dtype=torch.float16).cuda()
+    qs = _mats(fmt, Ms, K, seed=seed)
+    Wd = [torch.from_numpy(q).cuda() for q in qs]
+    outs = _grouped(fmt, Wd, Ms, K, x, ydt, flags=gq.GQ_GEMV_PDL)
     xo, xt = x_for_oracle(x)
-    for W, M, y in zip(Wd, Ms, outs):
-        rows = np.unique(np.concatenate([np.arange(0, M, 53), np.arange(15, M, 211), [M - 1]]))
-        Yr, bound = oracle.gemm_rows(Q40, W.cpu().numpy(), M, K, xo, rows.astype(np.int64), xt)
+    for q, M, y in zip(qs, Ms, outs):
+        rows = _every_group_rows(M)
+        Yr, bound = oracle.gemm_rows(fmt, q, M, K, xo, rows, xt)
         assert_product_close(y[:, torch.from_numpy(rows).cuda()], Yr, bound)
+
+
+@pytest.mark.parametrize("fmt", [Q40, KSB])
+def test_grouped_model_layer_shapes(fmt):
+    # one decoder layer of the whole-model stream (4 x 4096^2 and 3 x
+    # 11008x4096, 3088 row groups: the large-table configuration) with one x.
+    # K = 4096 makes both formats' rows whole 16-byte granules (2304 / 2208
+    # bytes), so the super-block case runs the compile-time word-offset
+    # branch of that configuration.
+    _large_table_case(fmt, [4096, 4096, 4096, 4096, 11008, 11008, 4096], 4096, seed=30000)
+
+
+def test_grouped_large_table_unaligned_q4_0_rows():
+    # the large-table configuration on Q4_0 rows that do not start on 16-byte
+    # boundaries: K = 2080 is 65 blocks, 1170-byte rows (1280 row groups)
+    _large_table_case(Q40, [4096] * 5, 2080, seed=41000, ydt=torch.float32)
+
+
+def test_grouped_large_table_unaligned_ksb_rows():
+    # super-block rows of K = 11008 (5934 bytes, starting at every even
+    # offset mod 16) on the large-table configuration (1376 row groups)
+    _large_table_case(KSB, [11008, 11008], 11008, seed=42000)
 
 
 @pytest.mark.parametrize("fmt", [Q40, KSB])
