@@ -80,6 +80,12 @@ def lib() -> ctypes.CDLL:
         L.orc_gemm_rows.argtypes = [ctypes.c_int, vp, i64, i64, vp, ctypes.c_int, i64,
                                     vp, i64, dp, dp]
         L.orc_num_threads.restype = ctypes.c_int
+        L.orc_tiled_bytes.argtypes = [ctypes.c_int, i64, i64]
+        L.orc_tiled_bytes.restype = i64
+        L.orc_repack.argtypes = [ctypes.c_int, vp, i64, i64, vp]
+        L.orc_repack.restype = ctypes.c_int
+        L.orc_unrepack.argtypes = [ctypes.c_int, vp, i64, i64, vp]
+        L.orc_unrepack.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -217,6 +223,33 @@ def gemm_rows(fmt: int, W, M: int, K: int, X, rows, xt: int | None = None):
     lib().orc_gemm_rows(fmt, _ptr(W), M, K, _ptr(X), _x_code(X, xt), B,
                         _ptr(rows), rows.size, _ptr(Y), _ptr(bound))
     return Y, bound
+
+
+def tiled_bytes(fmt: int, M: int, K: int) -> int:
+    """Bytes of the tiled storage of an M x K matrix (-1: K not a whole number
+    of units)."""
+    return int(lib().orc_tiled_bytes(fmt, M, K))
+
+
+def repack(fmt: int, W, M: int, K: int) -> np.ndarray:
+    """Canonical packed rows -> tiled storage (layout in gq_oracle.h)."""
+    W = np.ascontiguousarray(W, dtype=np.uint8).ravel()
+    n = tiled_bytes(fmt, M, K)
+    if n < 0:
+        raise ValueError("K must be a multiple of 64 (Q4_0) or 256 (ksb)")
+    out = np.zeros(n, dtype=np.uint8)
+    lib().orc_repack(fmt, _ptr(W), M, K, _ptr(out))
+    return out
+
+
+def unrepack(fmt: int, T, M: int, K: int) -> np.ndarray:
+    """Tiled storage -> canonical packed rows (the inverse of repack)."""
+    T = np.ascontiguousarray(T, dtype=np.uint8).ravel()
+    rb = q4_0_bytes(K) if fmt == FMT_Q4_0 else ksb_bytes(K)
+    out = np.zeros(M * rb, dtype=np.uint8)
+    if lib().orc_unrepack(fmt, _ptr(T), M, K, _ptr(out)) < 0:
+        raise ValueError("K must be a multiple of 64 (Q4_0) or 256 (ksb)")
+    return out
 
 
 def num_threads() -> int:

@@ -330,6 +330,117 @@ void orc_dequantize_ksb(const uint8_t* q, int64_t n, float* out) {
 }
 
 /* ------------------------------------------------------------------------ */
+/* Tiled storage: a byte permutation (layout in gq_oracle.h)                  */
+/* ------------------------------------------------------------------------ */
+
+static int64_t row_bytes(int fmt, int64_t K) {
+    return fmt == ORC_FMT_KSB ? K / KSB_BLOCK * KSB_BYTES : K / Q40_BLOCK * Q40_BYTES;
+}
+
+int64_t orc_tiled_bytes(int fmt, int64_t M, int64_t K) {
+    if (M < 0 || K < 0 || K % (fmt == ORC_FMT_KSB ? 256 : 64)) return -1;
+    return (M + 15) / 16 * 16 * row_bytes(fmt, K);
+}
+
+/* Visit every canonical byte once: call f(tiled offset, canonical offset)
+ * for each byte of each row group (rows past M give canonical offset -1). */
+typedef void (*visit_fn)(int64_t tiled, int64_t canon, const uint8_t* src, uint8_t* dst);
+
+static void visit_tiles(int fmt, int64_t M, int64_t K, visit_fn f, const uint8_t* src,
+                        uint8_t* dst) {
+    const int64_t rb = row_bytes(fmt, K);
+    const int64_t groups = (M + 15) / 16;
+    if (fmt == ORC_FMT_Q4_0) {
+        const int64_t nblk = K / 32;
+        for (int64_t g = 0; g < groups; ++g)
+            for (int64_t c0 = 0; c0 < nblk; c0 += 64) {
+                const int64_t nb = (nblk - c0 < 64) ? nblk - c0 : 64;
+                const int64_t tile = g * 16 * rb + c0 * 16 * 18;
+                for (int64_t u = 0; u < nb / 2; ++u) {
+                    for (int l = 0; l < 32; ++l) {
+                        const int gg = l / 4, t = l % 4;
+                        const int64_t rows[4] = {16 * g + gg, 16 * g + gg + 8, 16 * g + gg,
+                                                 16 * g + gg + 8};
+                        const int64_t blks[4] = {c0 + 2 * u, c0 + 2 * u, c0 + 2 * u + 1,
+                                                 c0 + 2 * u + 1};
+                        for (int w = 0; w < 4; ++w)
+                            for (int b = 0; b < 4; ++b) {
+                                const int64_t canon = rows[w] < M
+                                    ? rows[w] * rb + blks[w] * 18 + 2 + 4 * t + b : -1;
+                                f(tile + 512 * u + 16 * l + 4 * w + b, canon, src, dst);
+                            }
+                    }
+                    for (int r = 0; r < 16; ++r)
+                        for (int h = 0; h < 2; ++h)
+                            for (int b = 0; b < 2; ++b) {
+                                const int64_t row = 16 * g + r;
+                                const int64_t canon = row < M
+                                    ? row * rb + (c0 + 2 * u + h) * 18 + b : -1;
+                                f(tile + 256 * nb + 64 * u + 4 * r + 2 * h + b, canon, src, dst);
+                            }
+                }
+            }
+    } else {
+        const int64_t nsb = K / 256;
+        for (int64_t g = 0; g < groups; ++g)
+            for (int64_t c0 = 0; c0 < nsb; c0 += 8) {
+                const int64_t ns = (nsb - c0 < 8) ? nsb - c0 : 8;
+                const int64_t tile = g * 16 * rb + c0 * 16 * 138;
+                for (int64_t u = 0; u < 2 * ns; ++u) {
+                    const int64_t sb = c0 + u / 2;
+                    for (int l = 0; l < 32; ++l) {
+                        const int gg = l / 4, t = l % 4;
+                        for (int h = 0; h < 4; ++h) {
+                            const int64_t j = 4 * (u % 2) + h;
+                            for (int w = 0; w < 2; ++w) {
+                                const int64_t row = 16 * g + gg + 8 * w;
+                                for (int b = 0; b < 4; ++b) {
+                                    const int64_t canon = row < M
+                                        ? row * rb + sb * 138 + 10 + 16 * j + 4 * t + b : -1;
+                                    f(tile + 1024 * u + 32 * l + 8 * h + 4 * w + b, canon, src, dst);
+                                }
+                            }
+                        }
+                    }
+                    for (int r = 0; r < 16; ++r)
+                        for (int h = 0; h < 4; ++h) {
+                            const int64_t row = 16 * g + r;
+                            const int64_t canon = row < M
+                                ? row * rb + sb * 138 + 2 + 4 * (u % 2) + h : -1;
+                            f(tile + 2048 * ns + 64 * u + 4 * r + h, canon, src, dst);
+                        }
+                }
+                for (int64_t s = 0; s < ns; ++s)
+                    for (int r = 0; r < 16; ++r)
+                        for (int b = 0; b < 2; ++b) {
+                            const int64_t row = 16 * g + r;
+                            const int64_t canon = row < M ? row * rb + (c0 + s) * 138 + b : -1;
+                            f(tile + 2176 * ns + 32 * s + 2 * r + b, canon, src, dst);
+                        }
+            }
+    }
+}
+
+static void put_tiled(int64_t tiled, int64_t canon, const uint8_t* src, uint8_t* dst) {
+    dst[tiled] = canon >= 0 ? src[canon] : 0;
+}
+static void get_tiled(int64_t tiled, int64_t canon, const uint8_t* src, uint8_t* dst) {
+    if (canon >= 0) dst[canon] = src[tiled];
+}
+
+int orc_repack(int fmt, const uint8_t* W, int64_t M, int64_t K, uint8_t* out) {
+    if (orc_tiled_bytes(fmt, M, K) < 0) return -1;
+    visit_tiles(fmt, M, K, put_tiled, W, out);
+    return 0;
+}
+
+int orc_unrepack(int fmt, const uint8_t* T, int64_t M, int64_t K, uint8_t* out) {
+    if (orc_tiled_bytes(fmt, M, K) < 0) return -1;
+    visit_tiles(fmt, M, K, get_tiled, T, out);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Matrix products over the dequantized weights, fp64                        */
 /* ------------------------------------------------------------------------ */
 

@@ -90,6 +90,29 @@ void orc_gemm_rows(int fmt, const uint8_t* W, int64_t M, int64_t K,
                    const int64_t* rows, int64_t nrows,
                    double* Y, double* bound);
 
+/* Tiled storage (this library's own device layout; the pages have no
+ * counterpart): a permutation of the canonical bytes in which every tile of
+ * 16 rows x 64 Q4_0 blocks (16 rows x 8 super-blocks for ksb) is contiguous
+ * and arranged by the lanes that multiply it.  Rows are taken 16 at a time
+ * (rows past M are zero); tile (g, c) of row group g and K-tile c starts at
+ * byte g * 16 * rowbytes + c * 18432 (Q4_0) or c * 17664 (ksb); the last
+ * K-tile of a row holds the remaining blocks.  For lane l = 4 * gg + t
+ * (gg = 0..7, t = 0..3), "word t" of a block is its code bytes qs[4t..4t+3].
+ *   Q4_0 tile of nb blocks: unit u = blocks 2u, 2u+1.
+ *     codes at 512 u + 16 l: word t of block 2u of rows gg, gg+8, then of
+ *       block 2u+1 of rows gg, gg+8 (4 bytes each);
+ *     scales at 256 nb + 64 u + 4 r: d of blocks 2u, 2u+1 of row r.
+ *   ksb tile of ns super-blocks: unit u = half u % 2 of super-block u / 2
+ *     (sub-blocks j = 4 (u % 2) + h, h = 0..3).
+ *     codes at 1024 u + 32 l + 8 h: word t of sub-block j of rows gg, gg+8;
+ *     sub-scales at 2048 ns + 64 u + 4 r + h: q_j of row r;
+ *     super-scales at 2176 ns + 32 (u / 2) + 2 r: S of row r.
+ * Returns -1 when K is not a whole number of units (K % 64 for Q4_0,
+ * K % 256 for ksb). */
+int64_t orc_tiled_bytes(int fmt, int64_t M, int64_t K);
+int orc_repack(int fmt, const uint8_t* W, int64_t M, int64_t K, uint8_t* out);
+int orc_unrepack(int fmt, const uint8_t* T, int64_t M, int64_t K, uint8_t* out);
+
 /* Number of threads the parallel loops above use. */
 int orc_num_threads(void);
 

@@ -389,3 +389,63 @@ def test_gemm_rows_matches_full_product_and_bf16_input():
     rows = np.array([39, 0, 17])
     Yr, br = oracle.gemm_rows(oracle.FMT_Q4_0, q, M, K, Xbits, rows, xt=oracle.BF16)
     assert np.array_equal(Yr, Y[:, rows]) and np.array_equal(br, bound[:, rows])
+
+
+# ------------------------------------------------------------- tiled storage
+def test_tiled_layout_hand_worked_positions():
+    # each listed byte of the tiled storage holds the canonical byte worked out
+    # by hand from the layout definition (tests/golden/tiled_layout.txt)
+    rows = read_golden("tiled_layout.txt")
+    assert len(rows) == 24
+    for fmt, M, K, toff, coff in ((int(r[0]), int(r[1]), int(r[2]), int(r[3]), int(r[4]))
+                                  for r in rows):
+        rb = oracle.q4_0_bytes(K) if fmt == oracle.FMT_Q4_0 else oracle.ksb_bytes(K)
+        W = (np.arange(M * rb) * 7919 % 256).astype(np.uint8)
+        # make the probed canonical byte unique in the matrix
+        W[W == 255] = 254
+        W[coff] = 255
+        T = oracle.repack(fmt, W, M, K)
+        assert T[toff] == 255 and np.count_nonzero(T == 255) == 1, (fmt, M, K, toff, coff)
+
+
+@pytest.mark.parametrize("fmt,M,K", [(oracle.FMT_Q4_0, 16, 64), (oracle.FMT_Q4_0, 48, 4160),
+                                     (oracle.FMT_KSB, 32, 2304), (oracle.FMT_KSB, 16, 11008)])
+def test_tiled_is_a_byte_permutation(fmt, M, K):
+    # M a multiple of 16: same size, and the inverse restores every byte; with
+    # distinct 16-bit markers split over byte pairs, every tiled position is
+    # filled from exactly one canonical position
+    rb = oracle.q4_0_bytes(K) if fmt == oracle.FMT_Q4_0 else oracle.ksb_bytes(K)
+    assert oracle.tiled_bytes(fmt, M, K) == M * rb
+    rng = np.random.default_rng(M + K)
+    W = rng.integers(0, 256, M * rb, dtype=np.uint8)
+    T = oracle.repack(fmt, W, M, K)
+    assert np.array_equal(oracle.unrepack(fmt, T, M, K), W)
+    assert np.array_equal(np.sort(T), np.sort(W))
+
+
+@pytest.mark.parametrize("fmt,M,K", [(oracle.FMT_Q4_0, 17, 128), (oracle.FMT_KSB, 33, 512)])
+def test_tiled_ragged_rows_are_zero(fmt, M, K):
+    # rows past M in the last group of 16 are stored as zeros
+    rb = oracle.q4_0_bytes(K) if fmt == oracle.FMT_Q4_0 else oracle.ksb_bytes(K)
+    W = np.full(M * rb, 0xA5, dtype=np.uint8)
+    T = oracle.repack(fmt, W, M, K)
+    assert T.size == (M + 15) // 16 * 16 * rb
+    assert np.count_nonzero(T == 0xA5) == M * rb
+    assert np.count_nonzero(T == 0) == T.size - M * rb
+    assert np.array_equal(oracle.unrepack(fmt, T, M, K), W)
+
+
+def test_tiled_rejects_partial_units():
+    assert oracle.tiled_bytes(oracle.FMT_Q4_0, 16, 96) == -1
+    assert oracle.tiled_bytes(oracle.FMT_KSB, 16, 128) == -1
+
+
+def test_tiled_dequantizes_to_the_same_weights():
+    # a tiled matrix, turned back into rows, decodes to the canonical weights
+    M, K = 32, 2304
+    for fmt in (oracle.FMT_Q4_0, oracle.FMT_KSB):
+        w = synth.gaussian_weights(M, K, seed=5).numpy().ravel()
+        q, _ = oracle.quantize(fmt, w)
+        back = oracle.unrepack(fmt, oracle.repack(fmt, q, M, K), M, K)
+        assert np.array_equal(oracle.dequantize(fmt, back, M * K).view(np.uint32),
+                              oracle.dequantize(fmt, q, M * K).view(np.uint32))
