@@ -35,6 +35,7 @@ EXPORTS = (
     "gq_gemv_q4_0_grouped", "gq_gemv_ksb_grouped",
     "gq_gemm_workspace_bytes", "gq_gemm_q4_0", "gq_gemm_ksb",
     "gq_selftest_gemv_timeout", "gq_gemv_q4_0_noalloc", "gq_stream_read",
+    "gq_tiled_bytes", "gq_repack_q4_0", "gq_repack_ksb", "gq_gemv_q4_0_tiled", "gq_gemv_ksb_tiled",
 )
 
 _DTYPE_CODE = {torch.float32: GQ_F32, torch.float16: GQ_F16, torch.bfloat16: GQ_BF16}
@@ -94,6 +95,16 @@ def _load() -> ctypes.CDLL:
     L.gq_selftest_gemv_timeout.restype = c_int
     L.gq_stream_read.argtypes = [vp, ctypes.c_size_t, vp, vp]
     L.gq_stream_read.restype = c_int
+    L.gq_tiled_bytes.argtypes = [c_int, i64, i64]
+    L.gq_tiled_bytes.restype = ctypes.c_size_t
+    for name in ("gq_repack_q4_0", "gq_repack_ksb"):
+        f = getattr(L, name)
+        f.argtypes = [vp, i64, i64, vp, vp]
+        f.restype = c_int
+    for name in ("gq_gemv_q4_0_tiled", "gq_gemv_ksb_tiled"):
+        f = getattr(L, name)
+        f.argtypes = [vp, i64, i64, vp, c_int, vp, c_int, c_uint, vp, vp]
+        f.restype = c_int
     return L
 
 
@@ -374,3 +385,48 @@ def gq_stream_read(buf: torch.Tensor, sink: torch.Tensor | None = None,
     nbytes = buf.numel() * buf.element_size()
     _check(lib.gq_stream_read(_ptr(buf), nbytes, _ptr(sink), _stream(stream)), "gq_stream_read")
     return sink
+
+
+def gq_tiled_bytes(fmt: int, M: int, K: int) -> int:
+    """Bytes of the tiled storage of an M x K matrix (0 for unsupported K)."""
+    return int(lib.gq_tiled_bytes(int(fmt), int(M), int(K)))
+
+
+def gq_repack(fmt: int, W: torch.Tensor, M: int, K: int, out: torch.Tensor | None = None,
+              stream=None) -> torch.Tensor:
+    """Canonical packed rows (uint8 CUDA tensor) -> tiled storage (uint8)."""
+    n = gq_tiled_bytes(fmt, M, K)
+    if out is None:
+        out = torch.empty(n, dtype=torch.uint8, device=W.device)
+    name = "gq_repack_q4_0" if fmt == GQ_FMT_Q4_0 else "gq_repack_ksb"
+    _check(getattr(lib, name)(_ptr(W), int(M), int(K), _ptr(out), _stream(stream)), name)
+    return out
+
+
+def _gemv_tiled(name: str, T: torch.Tensor, M: int, K: int, x: torch.Tensor, y_dtype, out,
+                flags: int, dev_status, stream):
+    x1 = x.reshape(-1)
+    if x1.numel() != K:
+        raise ValueError(f"x has {x1.numel()} values, expected K={K}")
+    if x1.dtype not in _DTYPE_CODE or y_dtype not in _DTYPE_CODE:
+        raise TypeError("activations and outputs must be float32, float16 or bfloat16")
+    if out is None:
+        out = torch.empty((1, M), dtype=y_dtype, device=x1.device)
+    _check(getattr(lib, name)(_ptr(T), int(M), int(K), _ptr(x1), _DTYPE_CODE[x1.dtype],
+                              _ptr(out), _DTYPE_CODE[out.dtype], int(flags), _ptr(dev_status),
+                              _stream(stream)), name)
+    return out
+
+
+def gq_gemv_q4_0_tiled(T: torch.Tensor, M: int, K: int, x: torch.Tensor, y_dtype=torch.float16,
+                       out: torch.Tensor | None = None, flags: int = 0,
+                       dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y[1, M] = W_hat @ x for Q4_0 weights in tiled storage (x: K fp16 values)."""
+    return _gemv_tiled("gq_gemv_q4_0_tiled", T, M, K, x, y_dtype, out, flags, dev_status, stream)
+
+
+def gq_gemv_ksb_tiled(T: torch.Tensor, M: int, K: int, x: torch.Tensor, y_dtype=torch.float16,
+                      out: torch.Tensor | None = None, flags: int = 0,
+                      dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y[1, M] = W_hat @ x for super-block weights in tiled storage."""
+    return _gemv_tiled("gq_gemv_ksb_tiled", T, M, K, x, y_dtype, out, flags, dev_status, stream)

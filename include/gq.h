@@ -214,6 +214,60 @@ GQ_API gq_status gq_gemv_ksb_grouped(const gq_gemv_desc* mats, int count, int64_
                                      const void* x, int x_dtype, int64_t B, int y_dtype,
                                      unsigned flags, int* dev_status, void* stream);
 
+/* Tiled storage (no counterpart on the pages: a device layout of this
+ * library).  A byte permutation of the canonical rows in which every tile of
+ * 16 rows x 64 Q4_0 blocks (16 rows x 8 super-blocks for KSB) is contiguous
+ * and ordered by the lanes that multiply it, so that one bulk copy moves a
+ * whole pipeline stage and each lane's code words are aligned 16-byte reads.
+ * It holds the same bytes as the canonical rows (plus zero rows up to a
+ * multiple of 16), and is made once, e.g. when a model is loaded.
+ * Layout: rows are taken 16 at a time (row group g = rows 16g .. 16g+15, rows
+ * past M stored as zeros); tile (g, c) covers the K-tile c of group g and
+ * starts at byte g * 16 * R + c * 18432 (Q4_0) or c * 17664 (KSB), R the
+ * canonical row bytes; the last tile of a row holds the remaining blocks.
+ * For lane l = 4 gg + t (gg = 0..7, t = 0..3), "word t" of a block is its
+ * code bytes qs[4t .. 4t+3].
+ *   Q4_0 tile of nb blocks (nb even), unit u = blocks 2u, 2u+1:
+ *     at 512 u + 16 l: word t of block 2u of rows gg and gg+8, then of block
+ *       2u+1 of rows gg and gg+8 (4 bytes each);
+ *     at 256 nb + 64 u + 4 r: the FP16 scales of blocks 2u and 2u+1, row r.
+ *   KSB tile of ns super-blocks, unit u = sub-blocks j = 4 (u % 2) + h
+ *   (h = 0..3) of super-block u / 2:
+ *     at 1024 u + 32 l + 8 h: word t of sub-block j of rows gg and gg+8;
+ *     at 2048 ns + 64 u + 4 r + h: the INT8 sub-scale q_j of row r;
+ *     at 2176 ns + 32 (u / 2) + 2 r: the FP16 super-scale S of row r.
+ * gq_tiled_bytes: bytes of the tiled storage of an M x K matrix; 0 unless K
+ * is a multiple of 64 (Q4_0) or 256 (KSB).
+ * gq_repack_*: canonical rows W (M x K, as for gq_gemv_*) -> tiled storage
+ * `out` of gq_tiled_bytes(...) bytes; both 16-byte aligned, not overlapping.
+ * Asynchronous on `stream`; bad shapes give GQ_ERR_SHAPE. */
+GQ_API size_t gq_tiled_bytes(int fmt, int64_t M, int64_t K);
+GQ_API gq_status gq_repack_q4_0(const void* W, int64_t M, int64_t K, void* out, void* stream);
+GQ_API gq_status gq_repack_ksb(const void* W, int64_t M, int64_t K, void* out, void* stream);
+
+/* Batch-1 GEMV on tiled storage, y[m] = sum_k W_hat[m][k] * x[k] (the same
+ * product as gq_gemv_* with B = 1, computed from the tiled bytes): Q4_0
+ * chapter 4.3 and the K-quants post's step 5 for the decoded weights, the
+ * TurboQuant W4A8 post, section 2.3, for the memory-bound decode step.
+ *   T: gq_tiled_bytes(fmt, M, K) bytes from gq_repack_* (16-byte aligned).
+ *   K: a multiple of 64 (Q4_0) or 256 (KSB), at most 16384 (GQ_ERR_SHAPE).
+ *   x: K fp16 values (x_dtype must be GQ_F16, GQ_ERR_DTYPE otherwise).
+ *   y: M values of y_dtype (GQ_F16, GQ_BF16 or GQ_F32).
+ * Arithmetic: each 4-bit code enters the tensor core exactly (as an fp16
+ * subnormal c * 2^-24), the -8 offset enters as -8 * (block sum of x), and
+ * the fp32 MMA accumulation, the fp32 block sums of x and the fp32 sum over
+ * blocks round; the result is rounded once to y_dtype.  Non-finite
+ * activations give non-finite outputs.
+ * flags: 0 or GQ_GEMV_PDL (with PDL the kernel also stages its first tiles in
+ * tensor memory while the preceding kernel runs).  dev_status: optional,
+ * receives GQ_DEV_TIMEOUT if a pipeline wait ever gives up. */
+GQ_API gq_status gq_gemv_q4_0_tiled(const void* T, int64_t M, int64_t K, const void* x,
+                                    int x_dtype, void* y, int y_dtype, unsigned flags,
+                                    int* dev_status, void* stream);
+GQ_API gq_status gq_gemv_ksb_tiled(const void* T, int64_t M, int64_t K, const void* x, int x_dtype,
+                                   void* y, int y_dtype, unsigned flags, int* dev_status,
+                                   void* stream);
+
 /* Allocation-free variant (no counterpart on the pages): the batch-1 integer
  * tensor-core path of gq_gemv_q4_0 (fp16 x, B = 1) with its scratch -- the
  * per-CTA counts and partial sums, 33 KB -- in a static device array of the

@@ -221,3 +221,31 @@ def test_stream_read_validation():
     assert f(A + 8, 64, A, None) == ALIGN  # buffer off a 16-byte boundary
     assert f(A, 64, A + 2, None) == ALIGN  # sink off a 4-byte boundary
     assert f(None, 0, A, None) == GQ_OK  # nothing to read: no launch
+
+
+def test_tiled_sizes_and_validation():
+    Q, KS = gq.GQ_FMT_Q4_0, gq.GQ_FMT_KSB
+    assert gq.gq_tiled_bytes(Q, 16, 64) == 16 * 36
+    assert gq.gq_tiled_bytes(Q, 17, 11008) == 32 * 6192
+    assert gq.gq_tiled_bytes(KS, 4096, 11008) == 4096 * 5934
+    for fmt, bad_k in ((Q, 96), (Q, 32), (KS, 128), (KS, 2304 + 32)):
+        assert gq.gq_tiled_bytes(fmt, 16, bad_k) == 0
+    assert gq.gq_tiled_bytes(7, 16, 64) == 0 and gq.gq_tiled_bytes(Q, -1, 64) == 0
+    for name, k in (("gq_repack_q4_0", 64), ("gq_repack_ksb", 256)):
+        f = getattr(gq.lib, name)
+        assert f(A, -1, k, A, None) == INVALID
+        assert f(A, 16, k + 32, A, None) == SHAPE
+        assert f(A + 8, 16, k, A, None) == ALIGN
+        assert f(None, 16, k, A, None) == INVALID
+        assert f(A, 0, k, A, None) == GQ_OK  # nothing to do
+    for name, k in (("gq_gemv_q4_0_tiled", 64), ("gq_gemv_ksb_tiled", 256)):
+        f = getattr(gq.lib, name)
+        assert f(A, 16, k, A, gq.GQ_BF16, A, gq.GQ_F16, 0, None, None) == DTYPE
+        assert f(A, 16, k, A, gq.GQ_F16, A, 9, 0, None, None) == DTYPE
+        assert f(A, 16, k + 32, A, gq.GQ_F16, A, gq.GQ_F16, 0, None, None) == SHAPE
+        assert f(A, 16, 16384 + 256, A, gq.GQ_F16, A, gq.GQ_F16, 0, None, None) == SHAPE
+        assert f(A, 16, k, A, gq.GQ_F16, A, gq.GQ_F16, 2, None, None) == INVALID
+        assert f(A + 2, 16, k, A, gq.GQ_F16, A, gq.GQ_F16, 0, None, None) == ALIGN
+        assert f(A, 16, k, A, gq.GQ_F16, None, gq.GQ_F16, 0, None, None) == INVALID
+        assert f(A, -1, k, A, gq.GQ_F16, A, gq.GQ_F16, 0, None, None) == INVALID
+        assert f(A, 0, k, A, gq.GQ_F16, A, gq.GQ_F16, 0, None, None) == GQ_OK

@@ -114,6 +114,59 @@ def test_constant_codes_closed_form():
     assert torch.allclose(y.double().cpu(), want[:, None].expand(3, M), rtol=1e-5, atol=1e-4)
 
 
+# the batch-1 fp16 kernel: K a multiple of 64 (Q4_0) or 256 (super-blocks), up
+# to 16384; super-block rows of odd K / 256 are grouped by parity; ragged M
+@pytest.mark.parametrize("fmt,M,K", [
+    (Q40, 1, 64), (Q40, 3, 128), (Q40, 17, 1088), (Q40, 33, 16384), (Q40, 7, 16448),
+    (KSB, 1, 768), (KSB, 33, 256), (KSB, 47, 2816), (KSB, 65, 16384), (KSB, 31, 4352),
+])
+@pytest.mark.parametrize("flags", [0, 1])
+def test_batch1_fp16_shapes(fmt, M, K, flags):
+    check(fmt, M, K, 1, torch.float16, torch.float32, flags=flags)
+
+
+@pytest.mark.parametrize("fmt,M,K", [(Q40, 64, 16384), (KSB, 48, 11008), (Q40, 300, 11008),
+                                     (KSB, 129, 16384)])
+def test_batch1_tensor_memory_stash(fmt, M, K):
+    # few row groups over a long K: each CTA's share is more stages than the
+    # shared-memory ring holds, so with PDL the first stages go through
+    # tensor memory; three launches back to back on different matrices, each
+    # free to start while the previous one runs
+    qs = [packed(fmt, M, K, seed=M + K + i) for i in range(3)]
+    x = synth.activations(1, K, seed=K, dtype=torch.float16)
+    f = gq.gq_gemv_q4_0 if fmt == Q40 else gq.gq_gemv_ksb
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Wd = [torch.from_numpy(q).cuda() for q in qs]
+    xd = x.cuda()
+    ys = [f(W, M, K, xd, y_dtype=torch.float32, flags=gq.GQ_GEMV_PDL, dev_status=st) for W in Wd]
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    xo, xt = x_for_oracle(x)
+    for q, y in zip(qs, ys):
+        Y, bound = oracle.gemm(fmt, q, M, K, xo, xt)
+        assert_product_close(y, Y, bound)
+
+
+@pytest.mark.parametrize("fmt", [Q40, KSB])
+def test_batch1_extreme_activations(fmt):
+    # activations spanning the fp16 range: outliers near 3e4, values near 1e-3,
+    # fp16 subnormals, exact zeros and both signs
+    M, K = 96, 4096
+    q = packed(fmt, M, K)
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn((1, K), generator=g)
+    idx = torch.randperm(K, generator=g)
+    x[0, idx[:8]] = torch.tensor([3.0e4, -2.5e4, 1.2e4, -6.0e3, 900.0, -700.0, 4.0e3, -3.3e4])
+    x[0, idx[8:200]] *= 1e-3
+    x[0, idx[200:260]] = torch.randint(-1023, 1024, (60,), generator=g).float() * 2.0 ** -24
+    x[0, idx[260:300]] = 0.0
+    x = x.to(torch.float16)
+    for flags in (0, gq.GQ_GEMV_PDL):
+        y = run_gemv(fmt, q, M, K, x, torch.float32, flags)
+        Y, bound = oracle.gemm(fmt, q, M, K, *x_for_oracle(x))
+        assert_product_close(y, Y, bound)
+
+
 def test_misaligned_rows_large_k():
     # K = 11008 super-blocks give 5934-byte rows, so most rows start off a
     # 16-byte boundary; an offset view of W shifts them all
