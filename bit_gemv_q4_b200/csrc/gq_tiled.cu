@@ -461,10 +461,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tiled_kernel(const TArgs a) 
 #pragma unroll
         for (int i = 0; i < kStageWords; ++i) w[i] = 0u;
         const LaneOffs f = lane_offs<FMT>(sw, lane, ro);
-        if (nb == F::kPerTile)
-          tile_words<FMT, true>(static_cast<uint32_t>(s * kStageBytes), nb, sw, f, w);
-        else
-          tile_words<FMT, false>(static_cast<uint32_t>(s * kStageBytes), nb, sw, f, w);
+        tile_words<FMT, false>(static_cast<uint32_t>(s * kStageBytes), nb, sw, f, w);
         stash_store(tbase + tlane + static_cast<uint32_t>(k) * kStashCols, j, w);
       }
       tmem_wait_st();
@@ -497,38 +494,43 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tiled_kernel(const TArgs a) 
   for (int g0 = 0; g0 < ngc && ok; g0 += a.tgroups) {
     const int gn = min(a.tgroups, ngc - g0);
     float acc[2] = {0.f, 0.f};
-    for (int gi = g0; gi < g0 + gn && ok; ++gi) {
-      for (int c = 0, j = gi * a.ntiles; c < a.ntiles; ++c, ++j) {
-        const bool full_tile = c < a.ntiles - 1 || last_nb == F::kPerTile;
-        const int nb = full_tile ? F::kPerTile : last_nb;
-        uint32_t w[kStageWords];
-        const bool from_ring = j >= nstash;
-        const int s = j & (kRing - 1);
-        if (!from_ring) {
-          stash_load(tq, j, w);
-          tmem_wait_ld();
-        } else {
-          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (j / kRing) & 1u, a.budget))) {
-            ok = false;
-            break;
-          }
-          if (full_tile)
-            tile_words<FMT, true>(static_cast<uint32_t>(s * kStageBytes), nb, cw, f, w);
-          else
-            tile_words<FMT, false>(static_cast<uint32_t>(s * kStageBytes), nb, cw, f, w);
-        }
-        const uint32_t xb = xlane + c * 4096, cb = clane + c * 256;
-        if (full_tile)
-          stage_math<FMT, true>(w, acc, xb, cb, cw, nb, hi_row);
-        else
-          stage_math<FMT, false>(w, acc, xb, cb, cw, nb, hi_row);
-        if (from_ring) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[s]);
-        }
+    const int jend = (g0 + gn) * a.ntiles;
+    int j = g0 * a.ntiles, c = 0, gl = 0;
+    // a stage is done: on to the next tile, and past a row group's last tile
+    // its share goes to the table
+    auto next = [&]() {
+      if (++c == a.ntiles) {
+        if ((t & 1) == 0) tab[(gl * kCons + cw) * kRows + ro] = acc[0] + acc[1];
+        acc[0] = acc[1] = 0.f;
+        c = 0;
+        ++gl;
       }
-      if ((t & 1) == 0) tab[((gi - g0) * kCons + cw) * kRows + ro] = acc[0] + acc[1];
-      acc[0] = acc[1] = 0.f;
+    };
+    // stages held in tensor memory
+    for (const int je = min(jend, nstash); j < je; ++j) {
+      uint32_t w[kStageWords];
+      stash_load(tq, j, w);
+      tmem_wait_ld();
+      const uint32_t xb = xlane + c * 4096, cb = clane + c * 256;
+      stage_math<FMT, false>(w, acc, xb, cb, cw, c == a.ntiles - 1 ? last_nb : F::kPerTile, hi_row);
+      next();
+    }
+    // stages in the ring
+    for (; j < jend; ++j) {
+      const int s = j & (kRing - 1);
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (j / kRing) & 1u, a.budget))) {
+        ok = false;
+        break;
+      }
+      const uint32_t st = static_cast<uint32_t>(s * kStageBytes);
+      const uint32_t xb = xlane + c * 4096, cb = clane + c * 256;
+      const int nb = c == a.ntiles - 1 ? last_nb : F::kPerTile;
+      uint32_t w[kStageWords];
+      tile_words<FMT, false>(st, nb, cw, f, w);
+      stage_math<FMT, false>(w, acc, xb, cb, cw, nb, hi_row);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      next();
     }
     if (!ok) break;
     // every warp's share of the batch is in the table
