@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
         L.orc_gemm_rows.argtypes = [ctypes.c_int, vp, i64, i64, vp, ctypes.c_int, i64,
                                     vp, i64, dp, dp]
         L.orc_num_threads.restype = ctypes.c_int
+        L.orc_set_threads.argtypes = [ctypes.c_int]
+        L.orc_set_threads.restype = None
         L.orc_tiled_bytes.argtypes = [ctypes.c_int, i64, i64]
         L.orc_tiled_bytes.restype = i64
         L.orc_repack.argtypes = [ctypes.c_int, vp, i64, i64, vp]
@@ -254,3 +256,8 @@ def unrepack(fmt: int, T, M: int, K: int) -> np.ndarray:
 
 def num_threads() -> int:
     return int(lib().orc_num_threads())
+
+
+def set_threads(n: int) -> None:
+    """Threads of the oracle's parallel loops from now on (timing only)."""
+    lib().orc_set_threads(int(n))

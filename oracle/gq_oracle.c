@@ -512,3 +512,13 @@ int orc_num_threads(void) {
     return 1;
 #endif
 }
+
+/* Threads of the parallel loops that follow (timing runs only; results do
+ * not depend on it: every output is one thread's fp64 loop). */
+void orc_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

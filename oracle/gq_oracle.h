@@ -115,6 +115,7 @@ int orc_unrepack(int fmt, const uint8_t* T, int64_t M, int64_t K, uint8_t* out);
 
 /* Number of threads the parallel loops above use. */
 int orc_num_threads(void);
+void orc_set_threads(int n);
 
 #ifdef __cplusplus
 }

@@ -449,3 +449,19 @@ def test_tiled_dequantizes_to_the_same_weights():
         back = oracle.unrepack(fmt, oracle.repack(fmt, q, M, K), M, K)
         assert np.array_equal(oracle.dequantize(fmt, back, M * K).view(np.uint32),
                               oracle.dequantize(fmt, q, M * K).view(np.uint32))
+
+
+def test_thread_count_does_not_change_results():
+    # the timing runs change the oracle's thread count; every output is one
+    # thread's loop, so quantized bytes and products are the same bytes
+    w = synth.logstd_weights(96, 2048, seed=21).numpy().ravel()
+    x = synth.activations(3, 2048, seed=22, dtype=torch.float16).numpy()
+    res, n0 = [], oracle.num_threads()
+    for th in (1, 3, n0):
+        oracle.set_threads(th)
+        q4, _ = oracle.quantize(oracle.FMT_Q4_0, w)
+        qk, _ = oracle.quantize(oracle.FMT_KSB, w)
+        y, b = oracle.gemm(oracle.FMT_KSB, qk, 96, 2048, x)
+        res.append((q4.tobytes(), qk.tobytes(), y.tobytes(), b.tobytes()))
+    oracle.set_threads(n0)
+    assert res[0] == res[1] == res[2]
