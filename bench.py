@@ -1,17 +1,24 @@
 #!/usr/bin/env python3
 """Benchmark of the batch-1 Q4 GEMV decode stream on B200.
 
-Workload (one "step"): batch-1 GEMV y = W_hat x over the 4096x11008 weight
-shape in both Q4 formats and both orientations -- Q4_0 and super-block (ksb)
+Headline workload: batch-1 GEMV y = W_hat x over the 4096x11008 weight shape
+in both Q4 formats and both orientations -- Q4_0 and super-block (ksb)
 weights, M=4096 x K=11008 and M=11008 x K=4096 -- each over ``--copies``
 distinct copies of its packed matrix, launched back to back (CUDA graph,
-programmatic dependent launch).  A step streams ~1.6 GB of packed weights,
-far more than the 126 MB L2, so every GEMV reads cold weights.
+programmatic dependent launch), on both weight layouts the library serves:
+canonical rows (gq_gemv_*) and tiled storage (gq_gemv_*_tiled, made once by
+gq_repack_*).  A step is one pass over the four cases on both layouts; the
+copies rotate over far more than the 126 MB L2, so every GEMV reads cold
+weights.
 
-Metric: streamed-weight GB/s = packed weight bytes / device time.
+Metric: streamed-weight GB/s = packed weight bytes / device time, per case.
+``value`` is the worst of the four cases on the layout whose worst case is
+higher; the other cases, the other layout and the remaining hot-path rows
+(whole-model stream, batch 8, GEMM, quantize/dequantize, a plain read) are
+further keys of the same JSON line, each with its fraction of the measured
+peak.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--suite FILE]
 
 With N > 1 (torchrun), every rank runs the same workload on its own GPU
 (independent replicas: the path has no exchange step) and rank 0 prints the
@@ -20,6 +27,7 @@ aggregate over ranks with the max of the per-rank device times.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -33,30 +41,29 @@ sys.path.insert(0, ROOT)
 
 METRIC = "Q4 GEMV streamed-weight GB/s and % of HBM peak (4096x11008, batch 1)"
 CASES = [("q4_0", 4096, 11008), ("q4_0", 11008, 4096), ("ksb", 4096, 11008), ("ksb", 11008, 4096)]
+LAYOUTS = ("canonical", "tiled")
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
-# DRAM bytes (read + write) of one GEMV launch, the q4_0 4096x11008 case, from
-# one ncu capture (profiles/gemv_q4_0_4096x11008.md).  Reported only while the
-# GEMV sources hash to what was profiled; any change to the kernel makes it null.
-GEMV_TRAFFIC = {
-    "bytes": 25406976,
-    "sources": {
-        "bit_gemv_q4_b200/csrc/gq_gemv.cu": "2097710892fc724426aeafb75a26e0e3488edc2a224265dbdbaa265152e66880",
-        "bit_gemv_q4_b200/csrc/gq_device.cuh": "8eec6074ffd6e2337bf1ea2999f16285b22b3bca681a3cbf9c4acd0b821173c2",
-    },
-}
+# DRAM bytes (read + write) of one launch of each layout's kernel on the
+# q4_0 M=4096 K=11008 case, from one ncu capture of that kernel.  Reported
+# only while the kernel's sources hash to what was captured; a change to the
+# kernel makes it null until it is captured again.
+TRAFFIC = {}
 
 
-def gemv_traffic():
-    import hashlib
-    for rel, digest in GEMV_TRAFFIC["sources"].items():
+def traffic(layout):
+    entry = TRAFFIC.get(layout)
+    if not entry:
+        return None
+    for rel, digest in entry["sources"].items():
         try:
             with open(os.path.join(ROOT, rel), "rb") as f:
                 if hashlib.sha256(f.read()).hexdigest() != digest:
                     return None
         except OSError:
             return None
-    return GEMV_TRAFFIC["bytes"]
+    return entry["bytes"]
 
 
 def packed_bytes(fmt, M, K):
@@ -64,16 +71,17 @@ def packed_bytes(fmt, M, K):
 
 
 def measured_peaks():
+    """(HBM GB/s, bf16 TFLOP/s burst, source)."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
-        return float(p["hbm_gbs"]), "measured"
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
 # ----------------------------------------------------------------- clocks
-THROTTLE_BITS = {  # nvidia-smi clocks_event_reasons bit -> name
+THROTTLE_BITS = {  # clock-event reason bit -> name (NVML and nvidia-smi agree)
     0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
     0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
     0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
@@ -82,58 +90,92 @@ THROTTLE_BITS = {  # nvidia-smi clocks_event_reasons bit -> name
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clock and throttle reasons while running."""
+    """SM clock and clock-event reasons of this process's GPU (found by UUID),
+    read through NVML every `period` seconds while the run lasts; nvidia-smi
+    at 10 ms if NVML is unavailable."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, device_index: int, period: float = 0.005):
+        self.dev = device_index
+        self.period = period
+        self.samples = []  # (sm_mhz, sm_max_mhz, reason bits)
+        self.stop = threading.Event()
+        self.thread = None
         self.proc = None
-        self.lines = []
+        self.source = None
+
+    def _uuid(self):
+        import torch
+        return "GPU-" + str(torch.cuda.get_device_properties(self.dev).uuid)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu),
-                 "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(self._uuid())
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+
+            def loop():
+                while not self.stop.is_set():
+                    try:
+                        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        bits = reasons_fn(h)
+                        self.samples.append((float(sm), float(mx), int(bits)))
+                    except Exception:
+                        pass
+                    self.stop.wait(self.period)
+
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            self.source = f"NVML every {self.period * 1e3:.0f} ms"
         except Exception:
-            self.proc = None
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "--id=" + self._uuid(),
+                     "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+                     "--format=csv,noheader,nounits", "-lms", "10"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.thread = threading.Thread(target=self._read_smi, daemon=True)
+                self.thread.start()
+                self.source = "nvidia-smi every 10 ms"
+            except Exception:
+                self.proc = None
         return self
 
-    def _read(self):
+    def _read_smi(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            parts = [p.strip() for p in line.split(",")]
+            try:
+                self.samples.append((float(parts[0]), float(parts[1]), int(parts[2], 16)))
+            except (ValueError, IndexError):
+                continue
 
     def __exit__(self, *exc):
+        self.stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
-            self.t.join(timeout=2)
+        if self.thread is not None:
+            self.thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 3:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
-                bits = int(parts[2], 16)
-            except ValueError:
-                continue
+        busy = [s for s in self.samples if not (s[2] & 0x1)]
+        use = busy or self.samples
+        reasons = set()
+        for _, _, bits in use:
             for b, name in THROTTLE_BITS.items():
                 if bits & b and name != "gpu_idle":
                     reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": self.source}
+        return {"sm_mhz": statistics.median(s[0] for s in use),
+                "sm_max_mhz": max(s[1] for s in use), "reasons": sorted(reasons),
+                "samples": len(self.samples), "samples_busy": len(busy), "source": self.source}
 
 
 # ------------------------------------------------------------- distributed
@@ -180,40 +222,37 @@ def aggregate(units_per_rank: float, ms_per_rank: float, ws: int) -> tuple[float
 
 
 # --------------------------------------------------------------- our arm
-def build_gemv_set(gq, synth, copies, device, pdl=True):
-    """Packed weight copies, activations and outputs for the four cases."""
+def build_cases(gq, synth, copies, device):
+    """Packed weight copies on both layouts, activations and outputs for the
+    four headline cases."""
     import torch
     sets = []
     for ci, (fmt, M, K) in enumerate(CASES):
+        code = gq.GQ_FMT_Q4_0 if fmt == "q4_0" else gq.GQ_FMT_KSB
         w = synth.gaussian_weights(M, K, seed=100 + ci, device=device)
-        quant = gq.gq_quantize_q4_0 if fmt == "q4_0" else gq.gq_quantize_ksb
-        q = quant(w.view(-1))
+        q = (gq.gq_quantize_q4_0 if fmt == "q4_0" else gq.gq_quantize_ksb)(w.view(-1))
         del w
         nb = packed_bytes(fmt, M, K)
         Wc = torch.empty((copies, nb), dtype=torch.uint8, device=device)
         Wc.copy_(q.view(1, nb).expand(copies, nb))
+        Tc = torch.empty((copies, gq.gq_tiled_bytes(code, M, K)), dtype=torch.uint8, device=device)
+        for c in range(copies):
+            gq.gq_repack(code, Wc[c], M, K, out=Tc[c])
         x = synth.activations(1, K, seed=200 + ci, dtype=torch.float16, device=device)
         y = torch.empty((1, M), dtype=torch.float16, device=device)
-        gemv = gq.gq_gemv_q4_0 if fmt == "q4_0" else gq.gq_gemv_ksb
-        sets.append(dict(fmt=fmt, M=M, K=K, W=Wc, x=x, y=y, gemv=gemv, nbytes=nb, ws=None,
-                         kernels=1))
+        sets.append(dict(fmt=fmt, M=M, K=K, code=code, W=Wc, T=Tc, x=x, y=y, nbytes=nb,
+                         canonical=gq.gq_gemv_q4_0 if fmt == "q4_0" else gq.gq_gemv_ksb,
+                         tiled=gq.gq_gemv_q4_0_tiled if fmt == "q4_0" else gq.gq_gemv_ksb_tiled))
     torch.cuda.synchronize()
     return sets
 
 
-def gemv_workspace(gq, fmt, M, K, B, xdtype, device):
-    """A zeroed workspace for gq_gemv_* (None when the case needs none).  The
-    calls of one stream run in order, so they could share one."""
-    import torch
-    code = gq.GQ_FMT_Q4_0 if fmt == "q4_0" else gq.GQ_FMT_KSB
-    need = gq.gq_gemv_workspace_bytes(code, M, K, B, xdtype)
-    return torch.zeros(need, dtype=torch.uint8, device=device) if need else None
-
-
-def launch_case(gq, s, copies, flags):
+def launch_case(s, layout, copies, flags):
+    """`copies` GEMVs of one case, one per weight copy, through the C ABI."""
+    mats = s["W"] if layout == "canonical" else s["T"]
+    f = s[layout]
     for c in range(copies):
-        s["gemv"](s["W"][c], s["M"], s["K"], s["x"], y_dtype=s["y"].dtype, out=s["y"], flags=flags,
-                  workspace=s["ws"])
+        f(mats[c], s["M"], s["K"], s["x"], y_dtype=s["y"].dtype, out=s["y"], flags=flags)
 
 
 def capture(fn):
@@ -227,22 +266,231 @@ def capture(fn):
     return g
 
 
-def time_graph(g, steps, warmup, ws):
+def _timed(fn, reps, warmup=3):
+    """Device ms per call of fn(), CUDA events on the current stream."""
     import torch
     for _ in range(warmup):
-        g.replay()
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def _graph_ms(fn, reps):
+    """Device ms per replay of a CUDA graph of fn()."""
+    g = capture(fn)
+    ms = _timed(g.replay, reps)
+    del g
+    return ms
+
+
+def headline(args, sets, ws):
+    """K steps; each case of each layout is one CUDA graph of `copies` PDL
+    launches, replayed K times in a row between two events.  Returns
+    {(layout, case index): ms over the K replays (max over ranks)} and the
+    whole region's ms."""
+    import torch
+    import bit_gemv_q4_b200 as gq
+    copies, flags = args.copies, gq.GQ_GEMV_PDL
+    graphs = {}
+    for layout in LAYOUTS:
+        for i, s in enumerate(sets):
+            graphs[(layout, i)] = capture(lambda s=s, layout=layout: launch_case(s, layout, copies,
+                                                                                flags))
+    for g in graphs.values():
+        for _ in range(args.warmup):
+            g.replay()
+    ev = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for k in graphs}
     torch.cuda.synchronize()
     barrier(ws)
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for k, g in graphs.items():
+        ev[k][0].record()
+        for _ in range(args.steps):
+            g.replay()
+        ev[k][1].record()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms = {k: max_over_ranks(e[0].elapsed_time(e[1]), ws) for k, e in ev.items()}
+    total = max_over_ranks(t0.elapsed_time(t1), ws)
+    del graphs
+    return ms, total
+
+
+def e2e_run(args, sets, layout, ws):
+    """End to end through the public API with host buffers: every step copies
+    the four activation vectors from pinned host memory, calls gq_gemv_* once
+    per weight copy (eager, through the C ABI) and copies the four results
+    back into pinned host memory.  Device time of the whole loop."""
+    import torch
+    import bit_gemv_q4_b200 as gq
+    copies, flags = args.copies, gq.GQ_GEMV_PDL
+    hx = [s["x"].cpu().pin_memory() for s in sets]
+    hy = [torch.empty(s["y"].shape, dtype=s["y"].dtype).pin_memory() for s in sets]
+
+    def step():
+        for i, s in enumerate(sets):
+            s["x"].copy_(hx[i], non_blocking=True)
+        for s in sets:
+            launch_case(s, layout, copies, flags)
+        for i, s in enumerate(sets):
+            hy[i].copy_(s["y"], non_blocking=True)
+
+    steps = max(20, args.steps // 20)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(steps):
-        g.replay()
+        step()
     e1.record()
     torch.cuda.synchronize()
     barrier(ws)
-    return e0.elapsed_time(e1)
+    wbytes = sum(s["nbytes"] for s in sets) * copies
+    gbs, _ = aggregate(wbytes * steps / 1e9, e0.elapsed_time(e1), ws)
+    return {"value": round(gbs, 1), "unit": "GB/s",
+            "h2d_bytes_per_step": sum(s["K"] * 2 for s in sets),
+            "d2h_bytes_per_step": sum(s["M"] * 2 for s in sets),
+            "mode": f"eager gq_gemv_*{'_tiled' if layout == 'tiled' else ''} calls, "
+                    f"{len(sets) * copies} per step, pinned host copies in and out", "steps": steps}
+
+
+def extra_rows(gq, synth, dev, peak, bf16):
+    """The other hot-path rows, each on its own workload (CUDA events around
+    CUDA graphs; weight copies rotated past the L2 where the row is a stream)."""
+    import torch
+    out = {}
+
+    def quant(fmt, w):
+        return (gq.gq_quantize_q4_0 if fmt == "q4_0" else gq.gq_quantize_ksb)(w.reshape(-1))
+
+    def frac(gbs):
+        return round(gbs / peak, 4)
+
+    # whole-model weight stream: 32 layers x (4 x 4096^2 + 3 x 11008x4096), one x
+    ms_rows = {}
+    for fmt in ("q4_0", "ksb"):
+        shapes = ([(4096, 4096)] * 4 + [(11008, 4096)] * 3) * 32
+        mats, total = [], 0
+        for i, (M, K) in enumerate(shapes):
+            w = synth.gaussian_weights(M, K, seed=30000 + i, device=dev)
+            mats.append((quant(fmt, w), M, K))
+            total += mats[-1][0].numel()
+            del w
+        x = synth.activations(1, 4096, seed=9, dtype=torch.float16, device=dev)
+        ys = {M: torch.empty((1, M), dtype=torch.float16, device=dev) for M in (4096, 11008)}
+        f = gq.gq_gemv_q4_0 if fmt == "q4_0" else gq.gq_gemv_ksb
+        ms = _graph_ms(lambda: [f(qm, M, K, x, out=ys[M], flags=gq.GQ_GEMV_PDL)
+                                for qm, M, K in mats], 5)
+        fg = gq.gq_gemv_q4_0_grouped if fmt == "q4_0" else gq.gq_gemv_ksb_grouped
+        outs = [torch.empty((1, M), dtype=torch.float16, device=dev) for _, M, _ in mats]
+        Ws, Ms = [m[0] for m in mats], [m[1] for m in mats]
+        msg = _graph_ms(lambda: fg(Ws, Ms, 4096, x, outs=outs, flags=gq.GQ_GEMV_PDL), 5)
+        g1, g2 = total / (ms * 1e-3) / 1e9, total / (msg * 1e-3) / 1e9
+        ms_rows[fmt] = {"weight_bytes": total,
+                        "graph": {"ms": round(ms, 3), "gbs": round(g1, 1), "frac_of_peak": frac(g1),
+                                  "matrices_per_s": round(224 / (ms * 1e-3), 1)},
+                        "grouped": {"ms": round(msg, 3), "gbs": round(g2, 1),
+                                    "frac_of_peak": frac(g2),
+                                    "matrices_per_s": round(224 / (msg * 1e-3), 1)}}
+        del mats, Ws, outs
+        torch.cuda.empty_cache()
+    out["model_stream"] = dict(
+        workload="32 layers x (4 x 4096x4096 + 3 x 11008x4096) = 224 batch-1 GEMVs, x fp16; "
+                 "'graph': one CUDA graph of 224 PDL launches, 'grouped': one grouped call",
+        **ms_rows)
+
+    # batch 8 on the MLP shape, and the tensor-core GEMM on the same W
+    M, K = 11008, 4096
+    b8, gemm = {}, {}
+    for fmt in ("q4_0", "ksb"):
+        w = synth.gaussian_weights(M, K, seed=11, device=dev) if fmt == "q4_0" else \
+            synth.logstd_weights(M, K, seed=2, device=dev)
+        q = quant(fmt, w)
+        del w
+        nb = q.numel()
+        copies = 6
+        Wc = torch.empty((copies, nb), dtype=torch.uint8, device=dev)
+        Wc.copy_(q.view(1, nb).expand(copies, nb))
+        x8 = synth.activations(8, K, seed=8, dtype=torch.float16, device=dev)
+        y8 = torch.empty((8, M), dtype=torch.float16, device=dev)
+        f = gq.gq_gemv_q4_0 if fmt == "q4_0" else gq.gq_gemv_ksb
+        ms = _graph_ms(lambda: [f(Wc[i], M, K, x8, out=y8, flags=gq.GQ_GEMV_PDL)
+                                for i in range(copies)], 20) / copies
+        gbs = nb / (ms * 1e-3) / 1e9
+        b8[fmt] = {"us": round(ms * 1e3, 3), "gbs": round(gbs, 1), "frac_of_peak": frac(gbs),
+                   "tflops": round(2 * M * K * 8 / (ms * 1e-3) / 1e12, 3)}
+        fm = gq.gq_gemm_q4_0 if fmt == "q4_0" else gq.gq_gemm_ksb
+        gemm[fmt] = {}
+        for B in (16, 64, 256):
+            X = synth.activations(B, K, seed=12, dtype=torch.bfloat16, device=dev)
+            Y = torch.empty((B, M), dtype=torch.float32, device=dev)
+            wsp = torch.zeros(max(gq.gq_gemm_workspace_bytes(
+                gq.GQ_FMT_Q4_0 if fmt == "q4_0" else gq.GQ_FMT_KSB, M, K, B), 1),
+                dtype=torch.uint8, device=dev)
+            ms = _graph_ms(lambda: [fm(Wc[i], M, K, X, out=Y, workspace=wsp)
+                                    for i in range(copies)], 10) / copies
+            tf = 2.0 * M * K * B / (ms * 1e-3) / 1e12
+            gemm[fmt][str(B)] = {"us": round(ms * 1e3, 2), "tflops": round(tf, 1),
+                                 "frac_of_bf16_peak": round(tf / bf16, 4),
+                                 "weight_gbs": round(nb / (ms * 1e-3) / 1e9, 1)}
+        del Wc
+    out["batch8"] = dict(workload="W 11008x4096, X fp16 [8, 4096], Y fp16, 6 rotated copies", **b8)
+    out["gemm"] = dict(workload="W 11008x4096, X bf16 [B, 4096], Y fp32, 6 rotated copies; "
+                                "useful flops 2*M*K*B", **gemm)
+
+    # quantize and dequantize 1e9 weights ~ N(0, 0.02^2)
+    n = 1_000_000_000
+    w = synth.gaussian_weights(n // 8000, 8000, seed=4, frac=0.0, device=dev).view(-1)
+    qd = {}
+    for fmt, nbytes in (("q4_0", n // 32 * 18), ("ksb", n // 256 * 138)):
+        q = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        fq = gq.gq_quantize_q4_0 if fmt == "q4_0" else gq.gq_quantize_ksb
+        fd = gq.gq_dequantize_q4_0 if fmt == "q4_0" else gq.gq_dequantize_ksb
+        row = {}
+        for kind, fn in (("quantize", lambda: fq(w, out=q)), ("dequantize", lambda: fd(q, n, out=w))):
+            ms = _timed(fn, 5)
+            gbs = (4 * n + nbytes) / (ms * 1e-3) / 1e9
+            row[kind] = {"ms": round(ms, 3), "tbs": round(gbs / 1e3, 3), "frac_of_peak": frac(gbs),
+                         "gweights_per_s": round(n / (ms * 1e-3) / 1e9, 2)}
+        qd[fmt] = row
+        del q
+    del w
+    torch.cuda.empty_cache()
+    out["quantize_dequantize"] = dict(workload="1e9 fp32 weights <-> packed bytes; bytes = 4n + "
+                                               "packed", **qd)
+    return out
+
+
+def plain_read(args, sets, peak):
+    """The same weight copies read once each by a plain streaming-read
+    kernel (gq_stream_read), one launch per matrix, no PDL, same graph
+    method: a reference point for the GEMV launches, not a ceiling for them
+    (the GEMV chain uses PDL)."""
+    import torch
+    import bit_gemv_q4_b200 as gq
+    dev = sets[0]["W"].device
+    sink = torch.zeros(1, dtype=torch.int32, device=dev)
+    res = {}
+    for s in sets:
+        ms = _graph_ms(lambda s=s: [gq.gq_stream_read(s["W"][c], sink) for c in range(args.copies)],
+                       max(10, args.steps // 50)) / args.copies
+        gbs = s["nbytes"] / (ms * 1e-3) / 1e9
+        res[f"{s['fmt']} M={s['M']} K={s['K']}"] = {"gbs": round(gbs, 1),
+                                                     "frac_of_peak": round(gbs / peak, 4)}
+    return res
 
 
 def run_ours(args, rank, ws, local):
@@ -251,127 +499,95 @@ def run_ours(args, rank, ws, local):
     import synth
 
     dev = torch.device("cuda", torch.cuda.current_device())
+    peak, bf16, peak_src = measured_peaks()
     copies = args.copies
-    sets = build_gemv_set(gq, synth, copies, dev)
-    flags = gq.GQ_GEMV_PDL
-    wbytes_step = sum(s["nbytes"] for s in sets) * copies
-    algo_bytes_step = sum(s["nbytes"] + s["K"] * 2 + s["M"] * 2 for s in sets) * copies
-    launches_step = sum(s["kernels"] for s in sets) * copies
-
-    def step():
-        for s in sets:
-            launch_case(gq, s, copies, flags)
-
-    g = capture(step)
     with ClockSampler(local) as clk:
-        ms = time_graph(g, args.steps, args.warmup, ws)
-    gbs, ms_max = aggregate(wbytes_step * args.steps / 1e9, ms, ws)
-    ms_per_step = ms_max / args.steps
-    launches = launches_step * args.steps
+        sets = build_cases(gq, synth, copies, dev)
+        ms, total_ms = headline(args, sets, ws)
 
-    # per-case breakdown (same kernel, each case timed alone)
-    cases = {}
-    case_steps = max(20, args.steps // 10)
-    for s in sets:
-        gc = capture(lambda s=s: launch_case(gq, s, copies, flags))
-        mc = time_graph(gc, case_steps, args.warmup, ws)
-        us = mc * 1e3 / (case_steps * copies)
-        cases[f"{s['fmt']} M={s['M']} K={s['K']}"] = {
-            "gbs": round(s["nbytes"] / (us * 1e-6) / 1e9, 1), "us_per_gemv": round(us, 3)}
-        del gc
-    # same stream without programmatic dependent launch, for contrast
-    g_nopdl = capture(lambda: [launch_case(gq, s, copies, 0) for s in sets])
-    ms_nopdl = time_graph(g_nopdl, max(20, args.steps // 10), args.warmup, ws)
-    nopdl_gbs = wbytes_step * max(20, args.steps // 10) / (ms_nopdl / 1e3) / 1e9
-    del g_nopdl
+        per = {}
+        for layout in LAYOUTS:
+            per[layout] = {}
+            for i, s in enumerate(sets):
+                gemv_us = ms[(layout, i)] * 1e3 / (args.steps * copies)
+                gbs = s["nbytes"] / (gemv_us * 1e-6) / 1e9
+                per[layout][i] = (gbs, gemv_us)
+        worst = {lay: min(range(len(sets)), key=lambda i: per[lay][i][0]) for lay in LAYOUTS}
+        lead = max(LAYOUTS, key=lambda lay: per[lay][worst[lay]][0])
+        wi = worst[lead]
+        ws_case = sets[wi]
+        value = per[lead][wi][0] * ws  # whole job: every rank streams the same bytes
+        # the dominant kernel: the headline layout's kernel on the worst case
+        algo_launch = ws_case["nbytes"] + ws_case["K"] * 2 + ws_case["M"] * 2
+        achieved = algo_launch / (per[lead][wi][1] * 1e-6) / 1e9
 
-    # practical ceiling: the same weight copies read once each by a plain
-    # streaming-read kernel (gq_stream_read), one launch per matrix, same graph
-    sink = torch.zeros(1, dtype=torch.int32, device=dev)
-    g_read = capture(lambda: [gq.gq_stream_read(s["W"][c], sink) for s in sets
-                              for c in range(copies)])
-    read_steps = max(20, args.steps // 10)
-    ms_read = time_graph(g_read, read_steps, args.warmup, ws)
-    read_gbs = wbytes_step * read_steps / (ms_read / 1e3) / 1e9
-    del g_read
+        e2e = e2e_run(args, sets, lead, ws)
+        extras = extra_rows(gq, synth, dev, peak, bf16) if (rank == 0 and not args.no_extras) else {}
+        reads = plain_read(args, sets, peak) if rank == 0 else {}
+    barrier(ws)
 
-    # end to end through the public API with host buffers: each step copies
-    # the four activation vectors from pinned host memory, runs the step's
-    # GEMVs and reads the four results back into pinned host memory
-    hx = [s["x"].cpu().pin_memory() for s in sets]
-    hy = [torch.empty(s["y"].shape, dtype=s["y"].dtype).pin_memory() for s in sets]
+    def case_table(layout):
+        return {f"{s['fmt']} M={s['M']} K={s['K']}": {
+            "gbs": round(per[layout][i][0], 1), "us_per_gemv": round(per[layout][i][1], 3),
+            "frac_of_peak": round(per[layout][i][0] / peak, 4)} for i, s in enumerate(sets)}
 
-    def e2e_step():
-        for i, s in enumerate(sets):
-            s["x"].copy_(hx[i], non_blocking=True)
-        for s in sets:
-            launch_case(gq, s, copies, flags)
-        for i, s in enumerate(sets):
-            hy[i].copy_(s["y"], non_blocking=True)
-
-    e2e_steps = max(20, args.steps // 10)
-    try:
-        ge = capture(e2e_step)
-        ms_e2e = time_graph(ge, e2e_steps, args.warmup, ws)
-        e2e_mode = "CUDA graph with host copies"
-        del ge
-    except Exception:  # capture of pageable/pinned copies unsupported: eager
-        for _ in range(args.warmup):
-            e2e_step()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(e2e_steps):
-            e2e_step()
-        e1.record()
-        torch.cuda.synchronize()
-        ms_e2e = e0.elapsed_time(e1)
-        e2e_mode = "eager launches with host copies"
-    e2e_gbs, _ = aggregate(wbytes_step * e2e_steps / 1e9, ms_e2e, ws)
-    h2d = sum(s["K"] * 2 for s in sets)
-    d2h = sum(s["M"] * 2 for s in sets)
-    del g
-
-    peak, peak_src = measured_peaks()
-    per_gpu_algo_gbs = algo_bytes_step / (ms_per_step * 1e-3) / 1e9
+    all_bytes = sum(s["nbytes"] for s in sets) * copies
+    lead_ms = sum(ms[(lead, i)] for i in range(len(sets)))
+    kernel = {"canonical": "gemv_kernel (gq_gemv_q4_0 / gq_gemv_ksb)",
+              "tiled": "gemv_tiled_kernel (gq_gemv_q4_0_tiled / gq_gemv_ksb_tiled)"}
     result = {
-        "metric": METRIC, "value": round(gbs, 1), "unit": "GB/s", "n_gpus": ws,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f16", "data": "synthetic",
         "config": {
             "workload": ("batch-1 GEMV, Q4_0 and super-block weights, 4096x11008 in both "
                          "orientations (M=4096 K=11008 and M=11008 K=4096), x fp16, y fp16, "
-                         f"{copies} copies of each matrix per step"),
-            "weights_per_step_bytes": wbytes_step,
-            "l2": "inputs larger than L2 (weights rotated over %.2f GB per step)" % (wbytes_step / 1e9),
-            "launch": "CUDA graph, programmatic dependent launch",
+                         f"{copies} copies of each matrix; value = the worst of the four cases"),
+            "headline_case": f"{ws_case['fmt']} M={ws_case['M']} K={ws_case['K']}",
+            "headline_layout": lead,
+            "step": "one pass over the four cases on both layouts (canonical rows and tiled "
+                    f"storage), {2 * len(sets) * copies} GEMVs",
+            "l2": "inputs larger than L2 (each case rotates over %.2f GB of copies)"
+                  % (min(s["nbytes"] for s in sets) * copies / 1e9),
+            "launch": "CUDA graph per case and layout, programmatic dependent launch",
             "parallelism": "replicas" if ws > 1 else "single GPU",
         },
-        "frac_of_peak": round(gbs / ws / peak, 4),
-        "frac_of_nominal_8tbs": round(gbs / ws / 8000.0, 4),
-        "roofline": {"bound": "hbm", "achieved": round(per_gpu_algo_gbs, 1), "peak": peak,
-                     "peak_source": f"{peak_src} hbm_gbs", "unit": "GB/s",
-                     "frac": round(per_gpu_algo_gbs / peak, 4), "traffic": gemv_traffic(),
-                     "kernel": "gemv_kernel (all four cases)"},
-        "cases": cases,
-        "no_pdl_gbs": round(nopdl_gbs, 1),
-        "read_ceiling": {"gbs": round(read_gbs, 1), "frac_of_peak": round(read_gbs / peak, 4),
-                         "value_frac_of_ceiling": round(gbs / ws / read_gbs, 4),
-                         "what": "the same weight copies, one plain streaming-read launch "
-                                 "(gq_stream_read) per matrix, same CUDA graph"},
-        "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "mode": e2e_mode},
-        "gpu_launches": launches,
+        "frac_of_peak": round(value / ws / peak, 4),
+        "frac_of_nominal_8tbs": round(value / ws / 8000.0, 4),
+        "all_cases_gbs": round(all_bytes * args.steps / (lead_ms * 1e-3) / 1e9 * ws, 1),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "peak_source": f"{peak_src} hbm_gbs (burst copy)", "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic(lead),
+                     "kernel": kernel[lead] + f" on {ws_case['fmt']} M={ws_case['M']} "
+                                              f"K={ws_case['K']}",
+                     "algorithmic_bytes_per_launch": algo_launch},
+        "cases": {layout: case_table(layout) for layout in LAYOUTS},
+        "e2e": e2e,
+        "gpu_launches": 2 * len(sets) * copies * args.steps,
         "clocks": clk.summary(),
     }
+    if extras:
+        result.update(extras)
+    if reads:
+        result["plain_read"] = dict(
+            what="the same weight copies, one plain streaming-read launch (gq_stream_read) per "
+                 "matrix, no PDL: a reference point for the GEMV launches, not a ceiling", **reads)
     return result
 
 
 # ---------------------------------------------------- the oracle on the host
+def all_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
 class OracleSample:
-    """The four cases (one matrix each), quantized by the oracle; ``run``
-    times the oracle's product over them on the host cores."""
+    """The four headline cases (one matrix each), quantized by the oracle;
+    ``run`` times the oracle's product over them on the host cores."""
 
     def __init__(self):
         import oracle
@@ -387,9 +603,11 @@ class OracleSample:
             x = synth.activations(1, K, seed=200 + ci, dtype=torch.float16).numpy()
             self.mats.append((f, q, M, K, x, packed_bytes(fmt, M, K)))
 
-    def run(self, seconds: float):
+    def run(self, seconds: float, threads: int | None = None):
         """Whole passes over the four cases until `seconds` have passed;
         returns (GB/s of packed weights, threads, description)."""
+        threads = threads or all_cores()
+        self.oracle.set_threads(threads)
         done, nbytes, t0 = 0, 0, time.perf_counter()
         while True:
             f, q, M, K, x, nb = self.mats[done % len(self.mats)]
@@ -400,8 +618,96 @@ class OracleSample:
             if el >= seconds and done % len(self.mats) == 0:
                 break
         desc = (f"{done} oracle GEMVs ({done // len(self.mats)} pass(es) over the four cases, "
-                f"one matrix each) in {el:.1f} s")
-        return nbytes / el / 1e9, self.oracle.num_threads(), desc
+                f"one matrix each) in {el:.1f} s on {threads} thread(s)")
+        return nbytes / el / 1e9, threads, desc
+
+
+def _best(fn, reps):
+    best = None
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        fn()
+        el = time.perf_counter() - t0
+        best = el if best is None else min(best, el)
+    return best
+
+
+def oracle_configs():
+    """The oracle timed on each configuration's workload: 1 core and all
+    cores for the single-matrix configurations, all cores for the model
+    stream, the GEMM and quantize (bounded samples, scaled to the metric's
+    unit and named).  steady clock (perf_counter), best of 3 where small."""
+    import numpy as np
+    import oracle
+    import synth
+    import torch
+    oracle.build()
+    n_all = all_cores()
+    out = {"cores_available": n_all}
+
+    def both(fn, units, unit, reps=3):
+        r = {}
+        for th in (1, n_all):
+            oracle.set_threads(th)
+            el = _best(fn, reps)
+            r[f"{th}_core{'s' if th > 1 else ''}"] = round(units / el, 4)
+        return dict(unit=unit, **r)
+
+    # config 1: W fp32 256x1024 -> Q4_0, x fp32, y fp32
+    w = synth.gaussian_weights(256, 1024, seed=0).numpy().ravel()
+    q, _ = oracle.quantize(oracle.FMT_Q4_0, w)
+    x = np.random.default_rng(0).standard_normal(1024).astype(np.float32)
+    out["cfg1_gemv_256x1024"] = both(lambda: oracle.gemm(oracle.FMT_Q4_0, q, 256, 1024, x),
+                                     q.size / 1e9, "GB/s")
+    # config 2: 4096x4096 Q4_0, x fp16
+    w = synth.gaussian_weights(4096, 4096, seed=1).numpy().ravel()
+    q, _ = oracle.quantize(oracle.FMT_Q4_0, w)
+    x = synth.activations(1, 4096, seed=1, dtype=torch.float16).numpy()
+    out["cfg2_gemv_4096x4096_q4_0"] = both(lambda: oracle.gemm(oracle.FMT_Q4_0, q, 4096, 4096, x),
+                                           q.size / 1e9, "GB/s")
+    # config 3: 11008x4096 ksb, B = 1 and 8
+    w = synth.logstd_weights(11008, 4096, seed=2).numpy().ravel()
+    q, _ = oracle.quantize(oracle.FMT_KSB, w)
+    for B in (1, 8):
+        x = synth.activations(B, 4096, seed=3, dtype=torch.float16).numpy()
+        out[f"cfg3_gemv_11008x4096_ksb_B{B}"] = both(
+            lambda x=x, B=B: oracle.gemm(oracle.FMT_KSB, q, 11008, 4096, x), q.size / 1e9, "GB/s",
+            reps=1 if B > 1 else 3)
+    oracle.set_threads(n_all)
+    # config 4: the model stream, sampled as one matrix of each shape per format,
+    # weighted as a decoder layer (4 x 4096x4096 + 3 x 11008x4096)
+    for fmt, f in (("q4_0", oracle.FMT_Q4_0), ("ksb", oracle.FMT_KSB)):
+        x = synth.activations(1, 4096, seed=9, dtype=torch.float16).numpy()
+        t_layer, nb_layer = 0.0, 0
+        for i, (M, count) in enumerate(((4096, 4), (11008, 3))):
+            w = synth.gaussian_weights(M, 4096, seed=30000 + 4 * i).numpy().ravel()
+            qm = oracle.quantize(f, w)[0]
+            t_layer += count * _best(lambda: oracle.gemm(f, qm, M, 4096, x), 1)
+            nb_layer += count * qm.size
+        out[f"cfg4_model_stream_{fmt}"] = {
+            "unit": "GB/s", f"{n_all}_cores": round(nb_layer / t_layer / 1e9, 4),
+            "matrices_per_s": round(7 / t_layer, 2),
+            "sample": "one 4096x4096 and one 11008x4096 matrix, weighted 4:3 as in a layer"}
+    # config 5: GEMM on sampled rows; quantize 1e8 of the 1e9 weights
+    w = synth.gaussian_weights(11008, 4096, seed=11).numpy().ravel()
+    q, _ = oracle.quantize(oracle.FMT_Q4_0, w)
+    rows = np.arange(0, 11008, 11008 // 512, dtype=np.int64)[:512]
+    for B in (16, 64, 256):
+        X = synth.activations(B, 4096, seed=12, dtype=torch.bfloat16)
+        xo = X.view(torch.int16).numpy().view(np.uint16)
+        el = _best(lambda: oracle.gemm_rows(oracle.FMT_Q4_0, q, 11008, 4096, xo, rows,
+                                            oracle.BF16), 1)
+        out[f"cfg5_gemm_B{B}_q4_0"] = {"unit": "GFLOP/s",
+                                       f"{n_all}_cores": round(2 * rows.size * 4096 * B / el / 1e9, 3),
+                                       "sample": f"{rows.size} of the 11008 rows"}
+    n = 100_000_000
+    w = synth.gaussian_weights(n // 8000, 8000, seed=4, frac=0.0).numpy().ravel()
+    for fmt, f, per in (("q4_0", oracle.FMT_Q4_0, 18 / 32), ("ksb", oracle.FMT_KSB, 138 / 256)):
+        el = _best(lambda f=f: oracle.quantize(f, w), 1)
+        out[f"cfg5_quantize_{fmt}"] = {"unit": "GB/s",
+                                       f"{n_all}_cores": round(n * (4 + per) / el / 1e9, 3),
+                                       "sample": "1e8 of the 1e9 weights"}
+    return out
 
 
 def run_reference(args, rank, ws):
@@ -413,7 +719,7 @@ def run_reference(args, rank, ws):
     for _ in range(args.warmup):
         smp.run(0.0)
     vals, t0 = [], time.perf_counter()
-    cores = smp.oracle.num_threads()
+    cores = all_cores()
     for _ in range(args.steps):
         v, cores, _ = smp.run(0.0)
         vals.append(v)
@@ -435,188 +741,13 @@ def run_reference(args, rank, ws):
     }
 
 
-# ------------------------------------------------------------------ suite
-def _timed(fn, reps, warmup=3):
-    """Device ms per call of fn(), CUDA events on the current stream."""
-    import torch
-    for _ in range(warmup):
-        fn()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(reps):
-        fn()
-    e1.record()
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / reps
-
-
-def _graph_ms_per_launch(fn, launches, reps):
-    g = capture(fn)
-    ms = _timed(g.replay, reps)
-    del g
-    return ms / launches
-
-
-def run_suite(path):
-    """Every row of the hot path on its own workload; one JSON line per row."""
-    import torch
-    import bit_gemv_q4_b200 as gq
-    import synth
-    dev = torch.device("cuda", torch.cuda.current_device())
-    peak, peak_src = measured_peaks()
-    out = open(path, "w")
-
-    def emit(d):
-        out.write(json.dumps(d) + "\n")
-        out.flush()
-        print("suite:", json.dumps(d), file=sys.stderr, flush=True)
-
-    def quant(fmt, w):
-        return (gq.gq_quantize_q4_0 if fmt == "q4_0" else gq.gq_quantize_ksb)(w.view(-1))
-
-    # --- single GEMVs (decode shapes), cold weights, graph + PDL
-    for fmt, M, K, B, xdt, ydt, name, use_ws in (
-            ("q4_0", 256, 1024, 1, torch.float32, torch.float32, "tiny 256x1024 fp32", False),
-            ("q4_0", 4096, 4096, 1, torch.float16, torch.float16, "decode 4096x4096", False),
-            ("ksb", 11008, 4096, 1, torch.float16, torch.float16, "MLP 11008x4096 ksb B=1", False),
-            ("ksb", 11008, 4096, 8, torch.float16, torch.float16, "MLP 11008x4096 ksb B=8", False),
-            ("q4_0", 11008, 4096, 8, torch.float16, torch.float16, "MLP 11008x4096 q4_0 B=8", False),
-            # the batch-1 integer tensor-core path (workspace given), for comparison
-            ("q4_0", 4096, 4096, 1, torch.float16, torch.float16, "decode 4096x4096, integer path", True),
-            ("q4_0", 4096, 11008, 1, torch.float16, torch.float16, "4096x11008, integer path", True),
-            ("q4_0", 11008, 4096, 1, torch.float16, torch.float16, "11008x4096, integer path", True)):
-        w = synth.gaussian_weights(M, K, seed=7, device=dev)
-        q = quant(fmt, w)
-        del w
-        nb = q.numel()
-        copies = max(4, int(512e6 // nb))
-        Wc = torch.empty((copies, nb), dtype=torch.uint8, device=dev)
-        Wc.copy_(q.view(1, nb).expand(copies, nb))
-        x = synth.activations(B, K, seed=8, dtype=xdt, device=dev)
-        y = torch.empty((B, M), dtype=ydt, device=dev)
-        f = gq.gq_gemv_q4_0 if fmt == "q4_0" else gq.gq_gemv_ksb
-        wsp = gemv_workspace(gq, fmt, M, K, B, xdt, dev) if use_ws else None
-        ms = _graph_ms_per_launch(
-            lambda: [f(Wc[i], M, K, x, y_dtype=ydt, out=y, flags=gq.GQ_GEMV_PDL, workspace=wsp)
-                     for i in range(copies)],
-            copies, 20)
-        emit({"row": "gemv", "workload": name, "format": fmt, "M": M, "K": K, "B": B,
-              "us": round(ms * 1e3, 3), "weight_gbs": round(nb / (ms * 1e-3) / 1e9, 1),
-              "frac_of_peak": round(nb / (ms * 1e-3) / 1e9 / peak, 4),
-              "gflops": round(2 * M * K * B / (ms * 1e-3) / 1e9, 1)})
-        del Wc
-
-    # --- read ceiling of one launch: the same rotated copies of each headline
-    # matrix read once by a plain streaming-read kernel, graph of launches
-    sink = torch.zeros(1, dtype=torch.int32, device=dev)
-    for fmt, M, K in CASES:
-        nb = packed_bytes(fmt, M, K)
-        copies = max(4, int(512e6 // nb))
-        buf = torch.empty((copies, nb), dtype=torch.uint8, device=dev)
-        buf.fill_(7)
-        ms = _graph_ms_per_launch(lambda: [gq.gq_stream_read(buf[i], sink) for i in range(copies)],
-                                  copies, 20)
-        emit({"row": "read_ceiling", "workload": f"plain streaming read of one {fmt} {M}x{K} "
-              "matrix per launch", "bytes": nb, "us": round(ms * 1e3, 3),
-              "gbs": round(nb / (ms * 1e-3) / 1e9, 1),
-              "frac_of_peak": round(nb / (ms * 1e-3) / 1e9 / peak, 4)})
-        del buf
-
-    # --- whole-model weight stream: 32 layers x (4 x 4096^2 + 3 x 11008x4096)
-    for fmt in ("q4_0", "ksb"):
-        shapes = []
-        for layer in range(32):
-            shapes += [(4096, 4096)] * 4 + [(11008, 4096)] * 3
-        mats, total = [], 0
-        for i, (M, K) in enumerate(shapes):
-            w = synth.gaussian_weights(M, K, seed=30000 + i, device=dev)
-            mats.append((quant(fmt, w), M, K))
-            total += mats[-1][0].numel()
-            del w
-        x = synth.activations(1, 4096, seed=9, dtype=torch.float16, device=dev)
-        ys = {M: torch.empty((1, M), dtype=torch.float16, device=dev) for M in (4096, 11008)}
-        f = gq.gq_gemv_q4_0 if fmt == "q4_0" else gq.gq_gemv_ksb
-        wss = {M: None for M in (4096, 11008)}
-        ms = _graph_ms_per_launch(
-            lambda: [f(qm, M, K, x, out=ys[M], flags=gq.GQ_GEMV_PDL, workspace=wss[M])
-                     for qm, M, K in mats], 1, 5)
-        emit({"row": "model_stream", "workload": "32 layers x (4 x 4096x4096 + 3 x 11008x4096), "
-              "224 batch-1 GEMVs, one CUDA graph", "format": fmt, "weight_bytes": total,
-              "ms": round(ms, 3), "weight_gbs": round(total / (ms * 1e-3) / 1e9, 1),
-              "frac_of_peak": round(total / (ms * 1e-3) / 1e9 / peak, 4),
-              "matrices_per_s": round(224 / (ms * 1e-3), 1)})
-        # the same 224 products as one grouped call (one launch, x loaded once per CTA)
-        fg = gq.gq_gemv_q4_0_grouped if fmt == "q4_0" else gq.gq_gemv_ksb_grouped
-        outs = [torch.empty((1, M), dtype=torch.float16, device=dev) for _, M, _ in mats]
-        Ws, Ms = [m[0] for m in mats], [m[1] for m in mats]
-        ms = _graph_ms_per_launch(
-            lambda: fg(Ws, Ms, 4096, x, outs=outs, flags=gq.GQ_GEMV_PDL), 1, 5)
-        emit({"row": "model_stream_grouped", "workload": "32 layers x (4 x 4096x4096 + 3 x "
-              "11008x4096), 224 batch-1 GEMVs in one grouped call", "format": fmt,
-              "weight_bytes": total, "ms": round(ms, 3),
-              "weight_gbs": round(total / (ms * 1e-3) / 1e9, 1),
-              "frac_of_peak": round(total / (ms * 1e-3) / 1e9 / peak, 4),
-              "matrices_per_s": round(224 / (ms * 1e-3), 1)})
-        del Ws, outs
-        del mats
-        torch.cuda.empty_cache()
-
-    # --- tensor-core dequant-GEMM, W 11008x4096, X bf16 [B, 4096]
-    M, K = 11008, 4096
-    for fmt in ("q4_0", "ksb"):
-        w = synth.gaussian_weights(M, K, seed=11, device=dev)
-        q = quant(fmt, w)
-        del w
-        nb = q.numel()
-        copies = 6
-        Wc = torch.empty((copies, nb), dtype=torch.uint8, device=dev)
-        Wc.copy_(q.view(1, nb).expand(copies, nb))
-        f = gq.gq_gemm_q4_0 if fmt == "q4_0" else gq.gq_gemm_ksb
-        for B in (16, 64, 256):
-            X = synth.activations(B, K, seed=12, dtype=torch.bfloat16, device=dev)
-            Y = torch.empty((B, M), dtype=torch.float32, device=dev)
-            # one zeroed workspace for every call: a call leaves it ready for the next
-            code = gq.GQ_FMT_Q4_0 if fmt == "q4_0" else gq.GQ_FMT_KSB
-            wsp = torch.zeros(max(gq.gq_gemm_workspace_bytes(code, M, K, B), 1), dtype=torch.uint8,
-                              device=dev)
-            ms = _graph_ms_per_launch(
-                lambda: [f(Wc[i], M, K, X, out=Y, workspace=wsp) for i in range(copies)], copies, 10)
-            tf = 2.0 * M * K * B / (ms * 1e-3) / 1e12
-            emit({"row": "gemm", "workload": f"W {M}x{K} x X bf16 [{B},{K}], Y fp32",
-                  "format": fmt, "B": B, "us": round(ms * 1e3, 2), "tflops": round(tf, 1),
-                  "weight_gbs": round(nb / (ms * 1e-3) / 1e9, 1),
-                  "frac_of_bf16_peak": round(tf / 1615.2, 4),
-                  "note": "useful flops 2*M*K*B; the exact hi/lo split issues twice that"})
-        del Wc
-
-    # --- quantize and dequantize 1e9 weights ~ N(0, 0.02^2)
-    n = 1_000_000_000
-    w = synth.gaussian_weights(n // 8000, 8000, seed=4, frac=0.0, device=dev).view(-1)
-    for fmt, nbytes in (("q4_0", n // 32 * 18), ("ksb", n // 256 * 138)):
-        q = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-        fq = gq.gq_quantize_q4_0 if fmt == "q4_0" else gq.gq_quantize_ksb
-        ms = _timed(lambda: fq(w, out=q), 5)
-        emit({"row": "quantize", "workload": "1e9 fp32 weights", "format": fmt,
-              "ms": round(ms, 3), "gweights_per_s": round(n / (ms * 1e-3) / 1e9, 2),
-              "gbs": round((4 * n + nbytes) / (ms * 1e-3) / 1e9, 1),
-              "frac_of_peak": round((4 * n + nbytes) / (ms * 1e-3) / 1e9 / peak, 4)})
-        fd = gq.gq_dequantize_q4_0 if fmt == "q4_0" else gq.gq_dequantize_ksb
-        ms = _timed(lambda: fd(q, n, out=w), 5)
-        emit({"row": "dequantize", "workload": "1e9 weights to fp32", "format": fmt,
-              "ms": round(ms, 3), "gweights_per_s": round(n / (ms * 1e-3) / 1e9, 2),
-              "gbs": round((4 * n + nbytes) / (ms * 1e-3) / 1e9, 1),
-              "frac_of_peak": round((4 * n + nbytes) / (ms * 1e-3) / 1e9 / peak, 4)})
-        del q
-    out.close()
-
-
 def run_single(spec, launches, batch, flags, use_ws=False):
     """A few launches of one hot-path call (for profilers).  spec:
-    "gemv:q4_0:4096:11008" / "gemm:ksb:11008:4096" (distinct copies of one
-    matrix), "grouped:q4_0:<layers>" (the decoder-layer matrices
-    4 x 4096x4096 + 3 x 11008x4096 per layer in one grouped call), or
-    "quantize:ksb:<n>" / "dequantize:q4_0:<n>" (n weights)."""
+    "gemv:q4_0:4096:11008" / "tgemv:ksb:4096:11008" (canonical rows / tiled
+    storage) / "gemm:ksb:11008:4096" (distinct copies of one matrix),
+    "grouped:q4_0:<layers>" (the decoder-layer matrices 4 x 4096x4096 +
+    3 x 11008x4096 per layer in one grouped call), or "quantize:ksb:<n>" /
+    "dequantize:q4_0:<n>" (n weights)."""
     import torch
     import bit_gemv_q4_b200 as gq
     import synth
@@ -655,6 +786,7 @@ def run_single(spec, launches, batch, flags, use_ws=False):
         return
     kind, fmt, M, K = parts
     M, K = int(M), int(K)
+    code = gq.GQ_FMT_Q4_0 if fmt == "q4_0" else gq.GQ_FMT_KSB
     w = synth.gaussian_weights(M, K, seed=1, device=dev)
     q = (gq.gq_quantize_q4_0 if fmt == "q4_0" else gq.gq_quantize_ksb)(w.view(-1))
     del w
@@ -662,12 +794,23 @@ def run_single(spec, launches, batch, flags, use_ws=False):
     copies = 6
     Wc = torch.empty((copies, nb), dtype=torch.uint8, device=dev)
     Wc.copy_(q.view(1, nb).expand(copies, nb))
-    if kind == "gemv":
+    if kind in ("gemv", "tgemv"):
         x = synth.activations(batch, K, seed=2, dtype=torch.float16, device=dev)
-        f = gq.gq_gemv_q4_0 if fmt == "q4_0" else gq.gq_gemv_ksb
         y = torch.empty((batch, M), dtype=torch.float16, device=dev)
-        wsp = gemv_workspace(gq, fmt, M, K, batch, torch.float16, dev) if use_ws else None
-        run = lambda i: f(Wc[i % copies], M, K, x, out=y, flags=flags, workspace=wsp)
+        if kind == "tgemv":
+            Tc = torch.empty((copies, gq.gq_tiled_bytes(code, M, K)), dtype=torch.uint8, device=dev)
+            for c in range(copies):
+                gq.gq_repack(code, Wc[c], M, K, out=Tc[c])
+            del Wc
+            f = gq.gq_gemv_q4_0_tiled if fmt == "q4_0" else gq.gq_gemv_ksb_tiled
+            run = lambda i: f(Tc[i % copies], M, K, x, out=y, flags=flags)
+        else:
+            f = gq.gq_gemv_q4_0 if fmt == "q4_0" else gq.gq_gemv_ksb
+            wsp = None
+            if use_ws:
+                need = gq.gq_gemv_workspace_bytes(code, M, K, batch, torch.float16)
+                wsp = torch.zeros(need, dtype=torch.uint8, device=dev) if need else None
+            run = lambda i: f(Wc[i % copies], M, K, x, out=y, flags=flags, workspace=wsp)
     else:
         x = synth.activations(batch, K, seed=2, dtype=torch.bfloat16, device=dev)
         f = gq.gq_gemm_q4_0 if fmt == "q4_0" else gq.gq_gemm_ksb
@@ -682,17 +825,17 @@ def run_single(spec, launches, batch, flags, use_ws=False):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=4000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--copies", type=int, default=16)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="bounded sample of oracle work for cpu_baseline")
-    ap.add_argument("--suite", default=None,
-                    help="also measure every hot-path row; JSON lines written to this file")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the non-headline rows and the per-configuration oracle timings")
     ap.add_argument("--single", default=None,
                     help="profiling aid: launch one call a few times, e.g. gemv:q4_0:4096:11008, "
-                         "grouped:q4_0:2, quantize:ksb:268435456")
+                         "tgemv:q4_0:4096:11008, grouped:q4_0:2, quantize:ksb:268435456")
     ap.add_argument("--launches", type=int, default=4)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--flags", type=int, default=0)
@@ -713,8 +856,8 @@ def main():
                 v, cores, desc = OracleSample().run(args.cpu_seconds)
                 res["cpu_baseline"] = {"value": round(v, 3), "unit": "GB/s", "cores": cores,
                                        "kind": "oracle", "sample": desc}
-            if args.suite and rank == 0:
-                run_suite(args.suite)
+                if not args.no_extras:
+                    res["cpu_baselines"] = oracle_configs()
         if rank == 0 and res is not None:
             print(json.dumps(res), flush=True)
     finally:

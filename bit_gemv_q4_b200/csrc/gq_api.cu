@@ -24,6 +24,31 @@ int sm_count() {
   return n;
 }
 
+unsigned long long context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static const GetCurrent cur = []() -> GetCurrent {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<GetCurrent>(p);
+    return nullptr;
+  }();
+  static const GetId id = []() -> GetId {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<GetId>(p);
+    return nullptr;
+  }();
+  CUcontext c = nullptr;
+  unsigned long long v = 0;
+  if (!cur || !id || cur(&c) != CUDA_SUCCESS || !c || id(c, &v) != CUDA_SUCCESS) return 0;
+  return v;
+}
+
 EncodeTiled tensor_map_encoder() {
   // looked up once (a function-local static is initialized exactly once,
   // also when several threads arrive together)

@@ -775,14 +775,13 @@ gq_status gemm_entry(const void* W, int64_t M, int64_t K, const void* X, int xt,
 
   choose_stages(N, a.astages, a.xstages);
   const size_t smem = gemm_smem_bytes(N, a.astages, a.xstages);
-  thread_local int configured_dev = -1;  // per host thread (concurrent callers)
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
-  if (configured_dev != dev) {
+  thread_local unsigned long long configured_ctx = 0;  // per host thread and context
+  const unsigned long long ctx = context_id();
+  if (ctx == 0 || ctx != configured_ctx) {
     if (cudaFuncSetAttribute(gemm_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSmemBudget) != cudaSuccess)
       return GQ_ERR_CUDA;
-    configured_dev = dev;
+    configured_ctx = ctx;
   }
   return launch(gemm_kernel<FMT>, dim3(static_cast<unsigned>(a.sp.P)), dim3(kThreads), smem,
                 as_stream(stream), false, xmap, wmap, a);

@@ -159,7 +159,11 @@ __device__ __forceinline__ Unit unit_of(const GemvArgs& a, const Tbl& tbl, int g
 // holding (code - 8) as packed halves:
 //   r0 = (w[4t],    w[4t+2])     r1 = (w[4t+16], w[4t+18])
 //   r2 = (w[4t+1],  w[4t+3])     r3 = (w[4t+17], w[4t+19])
-// fp16: 0x6400 | n is 1024 + n; 0x6400 | (n << 4) is 1024 + 16n.
+// fp16: 0x6400 | n is 1024 + n; 0x6400 | (n << 4) is 1024 + 16n.  Placing
+// a 4-bit code in the mantissa of 1024.0 and subtracting the bias is the
+// integer-to-fp16 conversion published by Kim et al., "Who Says Elephants
+// Can't Run: Bringing Large Scale MoE Models into Cloud Scale Production"
+// (arXiv:2211.10017).
 __device__ __forceinline__ void decode_f16(uint32_t q, uint32_t r[4]) {
   const uint32_t q8 = __umulhi(q, 0x01000000u);  // q >> 8, on the FMA pipe
   uint32_t t0 = lop3_and_or(q, 0x000F000Fu, 0x64006400u);
@@ -788,13 +792,12 @@ gq_status launch_gemv(const GemvArgs& a, const Tbl& tbl, cudaStream_t stream, bo
   const size_t smem = gemv_smem_bytes(a.B, kTerms, a.win);
   // per host thread, so that concurrent callers (possibly on other devices)
   // never see each other's half-updated state
-  thread_local int configured_dev = -1;
+  thread_local unsigned long long configured_ctx = 0;
   thread_local size_t configured_smem = 0;
   thread_local size_t occ_smem = 0;
   thread_local int occupancy = 1;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
-  if (configured_dev != dev || smem > configured_smem) {
+  const unsigned long long ctx = context_id();
+  if (ctx == 0 || ctx != configured_ctx || smem > configured_smem) {
     // at least the common sizes, and always this launch's own requirement
     const size_t want = smem > gemv_smem_bytes(1, kTerms, 0) + kXSmemMax
                             ? smem
@@ -802,7 +805,7 @@ gq_status launch_gemv(const GemvArgs& a, const Tbl& tbl, cudaStream_t stream, bo
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(want)) != cudaSuccess)
       return GQ_ERR_CUDA;
-    configured_dev = dev;
+    configured_ctx = ctx;
     configured_smem = want;
     occ_smem = 0;
   }
@@ -1077,7 +1080,7 @@ GQ_API gq_status gq_gemv_q4_0_noalloc(const void* W, int64_t M, int64_t K, const
   if (!W || !x || !y) return GQ_ERR_INVALID_ARG;
   if (gq::misaligned16(W) || gq::misaligned16(x) || gq::misaligned16(y)) return GQ_ERR_ALIGNMENT;
   if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return GQ_ERR_ALIGNMENT;
-  if (!gq::i8_eligible(GQ_FMT_Q4_0, M, K, 1, GQ_F16, W)) return GQ_ERR_SHAPE;
+  if (!gq::i8_shape_ok(GQ_FMT_Q4_0, M, K, 1, GQ_F16, W)) return GQ_ERR_SHAPE;
   return gq::i8_gemv_noalloc(W, M, K, x, y, y_dtype, (flags & GQ_GEMV_PDL) != 0, dev_status,
                              gq::as_stream(stream));
 }

@@ -51,6 +51,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "gq.h"
 #include "gq_device.cuh"
@@ -578,12 +579,16 @@ __device__ __align__(256) uint8_t g_noalloc_scratch[kWsBytes];
 
 }  // namespace
 
-bool i8_eligible(int fmt, int64_t M, int64_t K, int64_t B, int xt, const void* W) {
+bool i8_shape_ok(int fmt, int64_t M, int64_t K, int64_t B, int xt, const void* W) {
   if (fmt != GQ_FMT_Q4_0 || B != 1 || xt != GQ_F16 || M <= 0) return false;
   if (K <= 0 || K % 256 != 0 || K / 32 > kMaxBlk) return false;  // whole 16-byte granules
   if (reinterpret_cast<uintptr_t>(W) & 15u) return false;
-  if (M > (1LL << 30) || sm_count() > kMaxCtas) return false;
+  if (M > (1LL << 30)) return false;
   return stages_for(static_cast<int>(K / 32)) >= 2;
+}
+
+bool i8_eligible(int fmt, int64_t M, int64_t K, int64_t B, int xt, const void* W) {
+  return i8_shape_ok(fmt, M, K, B, xt, W) && sm_count() <= kMaxCtas;
 }
 
 size_t i8_workspace_bytes(int64_t, int64_t) { return kWsBytes; }
@@ -612,14 +617,13 @@ gq_status i8_gemv(const void* W, int64_t M, int64_t K, const void* x, void* y, i
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return GQ_ERR_CUDA;
 
-  thread_local int configured_dev = -1;  // per host thread (concurrent callers)
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
-  if (configured_dev != dev) {
+  thread_local unsigned long long configured_ctx = 0;  // per host thread and context
+  const unsigned long long ctx = context_id();
+  if (ctx == 0 || ctx != configured_ctx) {
     if (cudaFuncSetAttribute(gemv_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBudget)) != cudaSuccess)
       return GQ_ERR_CUDA;
-    configured_dev = dev;
+    configured_ctx = ctx;
   }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   I8Args a;
@@ -642,16 +646,31 @@ gq_status i8_gemv(const void* W, int64_t M, int64_t K, const void* x, void* y, i
 
 namespace gq {
 
-// Address of the static scratch on the current device, looked up once per
-// device (the first call on a device should come before any stream capture).
+// Address of the static scratch in the calling thread's current context,
+// looked up once per context: a context created after another one was
+// destroyed (e.g. by cudaDeviceReset) holds the array at a new address.  The
+// first call in a context should come before any stream capture.
 static gq_status noalloc_scratch(uint8_t** out) {
-  static std::atomic<void*> addr[64];  // zero-initialized; same value from every thread
+  static std::mutex mu;
+  static unsigned long long ctx_of[64];  // zero: no context seen
+  static void* addr_of[64];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GQ_ERR_CUDA;
-  void* p = addr[dev].load(std::memory_order_relaxed);
-  if (!p) {
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GQ_ERR_CUDA;
-    addr[dev].store(p, std::memory_order_relaxed);
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return GQ_ERR_CUDA;
+  const unsigned long long ctx = context_id();
+  if (dev < 64 && ctx != 0) {
+    std::lock_guard<std::mutex> lock(mu);
+    if (ctx_of[dev] == ctx) {
+      *out = static_cast<uint8_t*>(addr_of[dev]);
+      return GQ_OK;
+    }
+  }
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GQ_ERR_CUDA;
+  const unsigned long long now = context_id();  // the lookup made a context current if none was
+  if (dev < 64 && now != 0) {
+    std::lock_guard<std::mutex> lock(mu);
+    ctx_of[dev] = now;
+    addr_of[dev] = p;
   }
   *out = static_cast<uint8_t*>(p);
   return GQ_OK;

@@ -14,6 +14,9 @@ namespace gq {
 // workspace: Q4_0, batch 1, fp16 x, K a multiple of 256 (rows of whole
 // 16-byte granules), W 16-byte aligned, and K short enough for the plan.
 bool i8_eligible(int fmt, int64_t M, int64_t K, int64_t B, int xt, const void* W);
+// The same test without the device's SM count (which only bounds the
+// scratch of gq_gemv_q4_0_noalloc, checked there).
+bool i8_shape_ok(int fmt, int64_t M, int64_t K, int64_t B, int xt, const void* W);
 
 // Workspace bytes of that path for an M x K matrix on the current device.
 size_t i8_workspace_bytes(int64_t M, int64_t K);

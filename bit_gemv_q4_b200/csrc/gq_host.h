@@ -22,6 +22,12 @@ inline int dtype_size(int t) { return t == GQ_F32 ? 4 : 2; }
 // Number of SMs of the current device (looked up once per device).
 int sm_count();
 
+// Process-unique ID of the calling thread's current CUDA context (0 if there
+// is none yet, or the driver cannot say).  Per-context state -- function
+// attributes, symbol addresses -- is keyed by it, so that it is set up again
+// when a context is destroyed and another one created.
+unsigned long long context_id();
+
 // cuTensorMapEncodeTiled from the driver (looked up once; null if missing).
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,

@@ -666,17 +666,16 @@ size_t tiled_smem(int K, int& tgroups, uint32_t& xf, uint32_t& xc, uint32_t& tab
 template <int FMT>
 gq_status launch_tiled(const TArgs& a0, int grid, size_t smem_bytes, bool pdl, cudaStream_t stream) {
   auto kern = gemv_tiled_kernel<FMT>;
-  thread_local int configured_dev = -1;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
-  if (configured_dev != dev) {
+  thread_local unsigned long long configured_ctx = 0;  // per host thread and context
+  const unsigned long long ctx = context_id();
+  if (ctx == 0 || ctx != configured_ctx) {
     // no layout exceeds the per-CTA budget, so one setting serves every call
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kCtaSmem)) != cudaSuccess ||
         cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return GQ_ERR_CUDA;
-    configured_dev = dev;
+    configured_ctx = ctx;
   }
   return launch(kern, dim3(grid), dim3(kThreads), smem_bytes, stream, pdl, a0);
 }

@@ -276,12 +276,14 @@ GQ_API gq_status gq_gemv_ksb_tiled(const void* T, int64_t M, int64_t K, const vo
  * on `stream` before each launch; the library allocates nothing.
  *   Arguments as for gq_gemv_q4_0 with x_dtype = GQ_F16, B = 1 and no
  *   workspace.  K must be a multiple of 256 and at most 14336
- *   (GQ_ERR_SHAPE otherwise); more SMs than the scratch covers (256) gives
+ *   (GQ_ERR_SHAPE otherwise); a launch wider than the scratch covers (more
+ *   than 256 CTAs, which needs a GPU of more than 256 SMs) gives
  *   GQ_ERR_WORKSPACE.
  *   The scratch is one per device: calls that may overlap (other streams,
  *   other host threads) race on it and must be serialised by the caller.
- *   The first call on a device looks the scratch up with
- *   cudaGetSymbolAddress; make it before capturing work into a graph. */
+ *   The first call in a CUDA context looks the scratch up with
+ *   cudaGetSymbolAddress; make it before capturing work into a graph.  A
+ *   context created later (e.g. after cudaDeviceReset) is looked up anew. */
 GQ_API gq_status gq_gemv_q4_0_noalloc(const void* W, int64_t M, int64_t K, const void* x,
                                       void* y, int y_dtype, unsigned flags, int* dev_status,
                                       void* stream);
