@@ -45,15 +45,24 @@ LAYOUTS = ("canonical", "tiled")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
-# DRAM bytes (read + write) of one launch of each layout's kernel on the
-# q4_0 M=4096 K=11008 case, from one ncu capture of that kernel.  Reported
-# only while the kernel's sources hash to what was captured; a change to the
-# kernel makes it null until it is captured again.
-TRAFFIC = {}
+# DRAM bytes (read + write) of one launch, from one ncu capture of that
+# kernel on that case (bench.py --single, a cold launch).  Reported only while
+# the kernel's sources hash to what was captured; a change to the kernel makes
+# it null until it is captured again.
+TRAFFIC = {
+    "canonical ksb 4096 11008": {"bytes": 24348672, "sources": {
+            "bit_gemv_q4_b200/csrc/gq_gemv.cu": "d8ae77602ecc157e27c7092587b20bf489427399d38b182d731f9d4a8e413880",
+            "bit_gemv_q4_b200/csrc/gq_gemv.h": "91b29c15fbd80ae3ad2435b203453a1ba1d4da29da52322e6e996adb97cd8ebe",
+            "bit_gemv_q4_b200/csrc/gq_device.cuh": "8eec6074ffd6e2337bf1ea2999f16285b22b3bca681a3cbf9c4acd0b821173c2"}},
+    "tiled q4_0 4096 11008": {"bytes": 25414656, "sources": {
+            "bit_gemv_q4_b200/csrc/gq_tiled.cu": "c77ec5b24e783a5b4e5ba052898913202c8c7cd175166b3c650409f02f9382e8",
+            "bit_gemv_q4_b200/csrc/gq_device.cuh": "8eec6074ffd6e2337bf1ea2999f16285b22b3bca681a3cbf9c4acd0b821173c2",
+            "bit_gemv_q4_b200/csrc/gq_tc.cuh": "b15f28de0672760637e15afae0059536e9c3acc85b1737d0e290acd10794f382"}},
+}
 
 
-def traffic(layout):
-    entry = TRAFFIC.get(layout)
+def traffic(layout, fmt, M, K):
+    entry = TRAFFIC.get(f"{layout} {fmt} {M} {K}")
     if not entry:
         return None
     for rel, digest in entry["sources"].items():
@@ -559,7 +568,8 @@ def run_ours(args, rank, ws, local):
         "all_cases_gbs": round(all_bytes * args.steps / (lead_ms * 1e-3) / 1e9 * ws, 1),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "peak_source": f"{peak_src} hbm_gbs (burst copy)", "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": traffic(lead),
+                     "frac": round(achieved / peak, 4),
+                     "traffic": traffic(lead, ws_case["fmt"], ws_case["M"], ws_case["K"]),
                      "kernel": kernel[lead] + f" on {ws_case['fmt']} M={ws_case['M']} "
                                               f"K={ws_case['K']}",
                      "algorithmic_bytes_per_launch": algo_launch},
