@@ -4,8 +4,9 @@
 Headline workload: batch-1 GEMV y = W_hat x over the 4096x11008 weight shape
 in both Q4 formats and both orientations -- Q4_0 and super-block (ksb)
 weights, M=4096 x K=11008 and M=11008 x K=4096 -- each over ``--copies``
-distinct copies of its packed matrix, launched back to back (CUDA graph,
-programmatic dependent launch), on both weight layouts the library serves:
+distinct copies of its packed matrix, launched back to back (a CUDA graph of
+``--chain`` launches cycling over the copies, programmatic dependent launch),
+on both weight layouts the library serves:
 canonical rows (gq_gemv_*) and tiled storage (gq_gemv_*_tiled, made once by
 gq_repack_*).  A step is one pass over the four cases on both layouts; the
 copies rotate over far more than the 126 MB L2, so every GEMV reads cold
@@ -256,12 +257,14 @@ def build_cases(gq, synth, copies, device):
     return sets
 
 
-def launch_case(s, layout, copies, flags):
-    """`copies` GEMVs of one case, one per weight copy, through the C ABI."""
+def launch_case(s, layout, launches, flags):
+    """`launches` GEMVs of one case through the C ABI, cycling over the
+    weight copies."""
     mats = s["W"] if layout == "canonical" else s["T"]
     f = s[layout]
-    for c in range(copies):
-        f(mats[c], s["M"], s["K"], s["x"], y_dtype=s["y"].dtype, out=s["y"], flags=flags)
+    for c in range(launches):
+        f(mats[c % mats.shape[0]], s["M"], s["K"], s["x"], y_dtype=s["y"].dtype, out=s["y"],
+          flags=flags)
 
 
 def capture(fn):
@@ -299,17 +302,17 @@ def _graph_ms(fn, reps):
 
 
 def headline(args, sets, ws):
-    """K steps; each case of each layout is one CUDA graph of `copies` PDL
-    launches, replayed K times in a row between two events.  Returns
-    {(layout, case index): ms over the K replays (max over ranks)} and the
-    whole region's ms."""
+    """K steps; each case of each layout is one CUDA graph of `chain` PDL
+    launches over the rotated copies, replayed K times in a row between two
+    events.  Returns {(layout, case index): ms over the K replays (max over
+    ranks)} and the whole region's ms."""
     import torch
     import bit_gemv_q4_b200 as gq
-    copies, flags = args.copies, gq.GQ_GEMV_PDL
+    chain, flags = args.chain, gq.GQ_GEMV_PDL
     graphs = {}
     for layout in LAYOUTS:
         for i, s in enumerate(sets):
-            graphs[(layout, i)] = capture(lambda s=s, layout=layout: launch_case(s, layout, copies,
+            graphs[(layout, i)] = capture(lambda s=s, layout=layout: launch_case(s, layout, chain,
                                                                                 flags))
     for g in graphs.values():
         for _ in range(args.warmup):
@@ -518,7 +521,7 @@ def run_ours(args, rank, ws, local):
         for layout in LAYOUTS:
             per[layout] = {}
             for i, s in enumerate(sets):
-                gemv_us = ms[(layout, i)] * 1e3 / (args.steps * copies)
+                gemv_us = ms[(layout, i)] * 1e3 / (args.steps * args.chain)
                 gbs = s["nbytes"] / (gemv_us * 1e-6) / 1e9
                 per[layout][i] = (gbs, gemv_us)
         worst = {lay: min(range(len(sets)), key=lambda i: per[lay][i][0]) for lay in LAYOUTS}
@@ -540,7 +543,7 @@ def run_ours(args, rank, ws, local):
             "gbs": round(per[layout][i][0], 1), "us_per_gemv": round(per[layout][i][1], 3),
             "frac_of_peak": round(per[layout][i][0] / peak, 4)} for i, s in enumerate(sets)}
 
-    all_bytes = sum(s["nbytes"] for s in sets) * copies
+    all_bytes = sum(s["nbytes"] for s in sets) * args.chain
     lead_ms = sum(ms[(lead, i)] for i in range(len(sets)))
     kernel = {"canonical": "gemv_kernel (gq_gemv_q4_0 / gq_gemv_ksb)",
               "tiled": "gemv_tiled_kernel (gq_gemv_q4_0_tiled / gq_gemv_ksb_tiled)"}
@@ -557,7 +560,8 @@ def run_ours(args, rank, ws, local):
             "headline_case": f"{ws_case['fmt']} M={ws_case['M']} K={ws_case['K']}",
             "headline_layout": lead,
             "step": "one pass over the four cases on both layouts (canonical rows and tiled "
-                    f"storage), {2 * len(sets) * copies} GEMVs",
+                    f"storage), {2 * len(sets) * args.chain} GEMVs",
+            "chain": f"{args.chain} GEMVs per CUDA graph, cycling over the {copies} copies",
             "l2": "inputs larger than L2 (each case rotates over %.2f GB of copies)"
                   % (min(s["nbytes"] for s in sets) * copies / 1e9),
             "launch": "CUDA graph per case and layout, programmatic dependent launch",
@@ -575,7 +579,7 @@ def run_ours(args, rank, ws, local):
                      "algorithmic_bytes_per_launch": algo_launch},
         "cases": {layout: case_table(layout) for layout in LAYOUTS},
         "e2e": e2e,
-        "gpu_launches": 2 * len(sets) * copies * args.steps,
+        "gpu_launches": 2 * len(sets) * args.chain * args.steps,
         "clocks": clk.summary(),
     }
     if extras:
@@ -839,6 +843,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--copies", type=int, default=16)
+    ap.add_argument("--chain", type=int, default=64,
+                    help="GEMVs per CUDA graph of a case (cycling over the copies)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="bounded sample of oracle work for cpu_baseline")
     ap.add_argument("--no-extras", action="store_true",
