@@ -55,8 +55,12 @@ TRAFFIC = {
             "bit_gemv_q4_b200/csrc/gq_gemv.cu": "d8ae77602ecc157e27c7092587b20bf489427399d38b182d731f9d4a8e413880",
             "bit_gemv_q4_b200/csrc/gq_gemv.h": "91b29c15fbd80ae3ad2435b203453a1ba1d4da29da52322e6e996adb97cd8ebe",
             "bit_gemv_q4_b200/csrc/gq_device.cuh": "8eec6074ffd6e2337bf1ea2999f16285b22b3bca681a3cbf9c4acd0b821173c2"}},
-    "tiled q4_0 4096 11008": {"bytes": 25414656, "sources": {
-            "bit_gemv_q4_b200/csrc/gq_tiled.cu": "c77ec5b24e783a5b4e5ba052898913202c8c7cd175166b3c650409f02f9382e8",
+    "tiled q4_0 4096 11008": {"bytes": 25415168, "sources": {
+            "bit_gemv_q4_b200/csrc/gq_tiled.cu": "27f50dc739335d5a567f47d03844e9c6e61ed2928678b31673212d2a9ccf6dfc",
+            "bit_gemv_q4_b200/csrc/gq_device.cuh": "8eec6074ffd6e2337bf1ea2999f16285b22b3bca681a3cbf9c4acd0b821173c2",
+            "bit_gemv_q4_b200/csrc/gq_tc.cuh": "b15f28de0672760637e15afae0059536e9c3acc85b1737d0e290acd10794f382"}},
+    "tiled ksb 4096 11008": {"bytes": 24358400, "sources": {
+            "bit_gemv_q4_b200/csrc/gq_tiled.cu": "27f50dc739335d5a567f47d03844e9c6e61ed2928678b31673212d2a9ccf6dfc",
             "bit_gemv_q4_b200/csrc/gq_device.cuh": "8eec6074ffd6e2337bf1ea2999f16285b22b3bca681a3cbf9c4acd0b821173c2",
             "bit_gemv_q4_b200/csrc/gq_tc.cuh": "b15f28de0672760637e15afae0059536e9c3acc85b1737d0e290acd10794f382"}},
 }

@@ -381,11 +381,16 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tiled_kernel(const TArgs a) 
   tc_fence_after();
   pdl_launch_dependents();
 
-  // this CTA's row groups g = blockIdx.x + i * gridDim.x, stage j = i * ntiles + c;
-  // stages [0, nstash) go through tensor memory, the rest through the ring
-  const int ngc = (a.ngroups - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
-                  static_cast<int>(gridDim.x);
-  const int ns = ngc * a.ntiles;
+  // This CTA's row groups g = blockIdx.x + i * gridDim.x; stage j is tile
+  // j % ntiles of group i = j / ntiles.  Stages [0, nstash) go through tensor
+  // memory, the rest through the ring.
+  const int nwhole = (a.ngroups - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                     static_cast<int>(gridDim.x);
+  const int ns = nwhole * a.ntiles;
+  auto stage_tile = [&](int j, int64_t& g, int& c) {  // stage j -> (row group, tile)
+    g = blockIdx.x + static_cast<int64_t>(j / a.ntiles) * gridDim.x;
+    c = j % a.ntiles;
+  };
   const int nstash = a.stash ? min(a.stash, max(0, ns - kRing)) : 0;
   const int last_nb = a.nblk - (a.ntiles - 1) * F::kPerTile;  // blocks in a row's last tile
 
@@ -395,25 +400,23 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tiled_kernel(const TArgs a) 
       const uint64_t pol = policy_evict_first();
       int issued = 0;
       bool ok = true;
-      int s = 0, c = 0;
+      int s = 0;
       uint32_t ph = 0;
-      const uint8_t* grp = a.T + static_cast<int64_t>(blockIdx.x) * a.group_bytes;
-      const int64_t gstep = static_cast<int64_t>(gridDim.x) * a.group_bytes;
       for (int j = 0; j < ns; ++j) {
         if (!mbar_wait(&empty[s], ph ^ 1u, a.budget)) {
           ok = false;
           break;
         }
+        int64_t g;
+        int c;
+        stage_tile(j, g, c);
         const int nb = (c == a.ntiles - 1) ? last_nb : F::kPerTile;
         const uint32_t bytes = static_cast<uint32_t>(nb * kRows * F::kBlkB);
         mbar_arrive_expect_tx(&full[s], bytes);
-        bulk_g2s(smem + s * kStageBytes, grp + static_cast<int64_t>(c) * F::kTileBytes, bytes,
+        bulk_g2s(smem + s * kStageBytes,
+                 a.T + g * a.group_bytes + static_cast<int64_t>(c) * F::kTileBytes, bytes,
                  &full[s], pol);
         ++issued;
-        if (++c == a.ntiles) {
-          c = 0;
-          grp += gstep;
-        }
         if (++s == kRing) {
           s = 0;
           ph ^= 1u;
@@ -452,7 +455,9 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tiled_kernel(const TArgs a) 
         ok = false;
         break;
       }
-      const int c = j % a.ntiles;
+      int64_t g_unused;
+      int c;
+      stage_tile(j, g_unused, c);
       const int nb = (c == a.ntiles - 1) ? last_nb : F::kPerTile;
 #pragma unroll 1
       for (int k = 0; k < kSiblings; ++k) {
@@ -491,36 +496,31 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tiled_kernel(const TArgs a) 
   const uint32_t clane = a.xc_off + F::kUnitBlk * cw * 4;
   float* tab = reinterpret_cast<float*>(smem + a.tab_off);
   uint32_t bar_uses = 0;
-  for (int g0 = 0; g0 < ngc && ok; g0 += a.tgroups) {
-    const int gn = min(a.tgroups, ngc - g0);
-    float acc[2] = {0.f, 0.f};
-    const int jend = (g0 + gn) * a.ntiles;
-    int j = g0 * a.ntiles, c = 0, gl = 0;
-    // a stage is done: on to the next tile, and past a row group's last tile
-    // its share goes to the table
-    auto next = [&]() {
-      if (++c == a.ntiles) {
-        if ((t & 1) == 0) tab[(gl * kCons + cw) * kRows + ro] = acc[0] + acc[1];
-        acc[0] = acc[1] = 0.f;
-        c = 0;
-        ++gl;
-      }
-    };
-    // stages held in tensor memory
-    for (const int je = min(jend, nstash); j < je; ++j) {
+  float acc[2] = {0.f, 0.f};
+  // a warp's share of a row group goes to table slot `slot`
+  auto flush = [&](int slot) {
+    if ((t & 1) == 0) tab[(slot * kCons + cw) * kRows + ro] = acc[0] + acc[1];
+    acc[0] = acc[1] = 0.f;
+  };
+  // stages [j, jend), the first being tile c; each group's share goes to the
+  // next table slot
+  auto run = [&](int j, const int jend, int c, int slot) {
+    for (const int je = min(jend, nstash); j < je; ++j) {  // in tensor memory
       uint32_t w[kStageWords];
       stash_load(tq, j, w);
       tmem_wait_ld();
       const uint32_t xb = xlane + c * 4096, cb = clane + c * 256;
       stage_math<FMT, false>(w, acc, xb, cb, cw, c == a.ntiles - 1 ? last_nb : F::kPerTile, hi_row);
-      next();
+      if (++c == a.ntiles) {
+        flush(slot++);
+        c = 0;
+      }
     }
-    // stages in the ring
-    for (; j < jend; ++j) {
+    for (; j < jend; ++j) {  // in the ring
       const int s = j & (kRing - 1);
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (j / kRing) & 1u, a.budget))) {
         ok = false;
-        break;
+        return;
       }
       const uint32_t st = static_cast<uint32_t>(s * kStageBytes);
       const uint32_t xb = xlane + c * 4096, cb = clane + c * 256;
@@ -530,38 +530,42 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tiled_kernel(const TArgs a) 
       stage_math<FMT, false>(w, acc, xb, cb, cw, nb, hi_row);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
-      next();
+      if (++c == a.ntiles) {
+        flush(slot++);
+        c = 0;
+      }
     }
-    if (!ok) break;
-    // every warp's share of the batch is in the table
+  };
+  // every warp's shares are in the table
+  auto table_barrier = [&]() {
     __syncwarp();
     if (lane == 0) mbar_arrive(red_bar);
-    if (!__all_sync(0xFFFFFFFFu, mbar_wait(red_bar, bar_uses & 1u, a.budget))) {
-      ok = false;
-      break;
-    }
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(red_bar, bar_uses & 1u, a.budget))) ok = false;
     ++bar_uses;
-    for (int gb = cw; gb < gn; gb += kCons) {
-      if (lane < kRows) {
-        float v = 0.f;
+  };
+  // the sum of slot `slot` over the warps (lanes 0..15: one row each): the
+  // output of row group g
+  auto finish = [&](int slot, int64_t g) {
+    float v = 0.f;
 #pragma unroll
-        for (int ww = 0; ww < kCons; ++ww) v += tab[(gb * kCons + ww) * kRows + lane];
-        const int64_t row =
-            (static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(g0 + gb) * gridDim.x) * kRows +
-            lane;
-        if (row < a.M) store_elem(a.y, row, v * 16777216.0f, a.ytype);  // * 2^24
-      }
-    }
-    if (g0 + gn < ngc) {
-      // the next batch reuses the table once every warp has read it
-      __syncwarp();
-      if (lane == 0) mbar_arrive(red_bar);
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(red_bar, bar_uses & 1u, a.budget))) {
-        ok = false;
-        break;
-      }
-      ++bar_uses;
-    }
+    for (int ww = 0; ww < kCons; ++ww) v += tab[(slot * kCons + ww) * kRows + lane];
+    const int64_t row = g * kRows + lane;
+    if (row < a.M) store_elem(a.y, row, v * 16777216.0f, a.ytype);  // * 2^24
+  };
+
+  int j = 0;
+  // row groups, in batches of tgroups
+  for (int w0 = 0; w0 < nwhole && ok; w0 += a.tgroups) {
+    const int gn = min(a.tgroups, nwhole - w0);
+    run(j, j + gn * a.ntiles, 0, 0);
+    j += gn * a.ntiles;
+    if (!ok) break;
+    table_barrier();
+    if (!ok) break;
+    if (lane < kRows)
+      for (int sl = cw; sl < gn; sl += kCons)
+        finish(sl, blockIdx.x + static_cast<int64_t>(w0 + sl) * gridDim.x);
+    if (w0 + gn < nwhole) table_barrier();  // the next batch reuses the table
   }
   if (!ok && lane == 0) report(a.dev_status, GQ_DEV_TIMEOUT);
 
