@@ -155,3 +155,19 @@ def test_tiled_gemv_table_batches(fmt):
     Y, bound = oracle.gemm(fmt, q, M, K, *x_for_oracle(x))
     for flags in (0, gq.GQ_GEMV_PDL):
         assert_product_close(run(fmt, T, M, K, x, torch.float32, flags), Y, bound)
+
+
+@pytest.mark.parametrize("fmt", [Q40, KSB])
+@pytest.mark.parametrize("bad", [float("inf"), float("-inf"), float("nan")])
+def test_tiled_gemv_nonfinite_activation(fmt, bad):
+    # one non-finite activation reaches every output row: each row multiplies
+    # it by a decoded weight, and the block's -8 * sum(x) correction carries
+    # it even where the code is 8 (weight zero)
+    M, K = 48, 2048
+    q = packed(fmt, M, K)
+    x = synth.activations(1, K, seed=4, dtype=torch.float16)
+    x[0, 777] = bad
+    T = tiled(fmt, q, M, K)
+    for flags in (0, gq.GQ_GEMV_PDL):
+        y = run(fmt, T, M, K, x, torch.float32, flags)
+        assert not bool(torch.isfinite(y).any())
