@@ -36,6 +36,7 @@ EXPORTS = (
     "gq_gemm_workspace_bytes", "gq_gemm_q4_0", "gq_gemm_ksb",
     "gq_selftest_gemv_timeout", "gq_gemv_q4_0_noalloc", "gq_stream_read",
     "gq_tiled_bytes", "gq_repack_q4_0", "gq_repack_ksb", "gq_gemv_q4_0_tiled", "gq_gemv_ksb_tiled",
+    "gq_gemv_q4_0_tiled_grouped", "gq_gemv_ksb_tiled_grouped",
 )
 
 _DTYPE_CODE = {torch.float32: GQ_F32, torch.float16: GQ_F16, torch.bfloat16: GQ_BF16}
@@ -104,6 +105,10 @@ def _load() -> ctypes.CDLL:
     for name in ("gq_gemv_q4_0_tiled", "gq_gemv_ksb_tiled"):
         f = getattr(L, name)
         f.argtypes = [vp, i64, i64, vp, c_int, vp, c_int, c_uint, vp, vp]
+        f.restype = c_int
+    for name in ("gq_gemv_q4_0_tiled_grouped", "gq_gemv_ksb_tiled_grouped"):
+        f = getattr(L, name)
+        f.argtypes = [vp, c_int, i64, vp, c_int, c_int, c_uint, vp, vp]
         f.restype = c_int
     return L
 
@@ -430,3 +435,41 @@ def gq_gemv_ksb_tiled(T: torch.Tensor, M: int, K: int, x: torch.Tensor, y_dtype=
                       dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """y[1, M] = W_hat @ x for super-block weights in tiled storage."""
     return _gemv_tiled("gq_gemv_ksb_tiled", T, M, K, x, y_dtype, out, flags, dev_status, stream)
+
+
+def _gemv_tiled_grouped(name: str, Ts, Ms, K: int, x: torch.Tensor, y_dtype, outs, flags: int,
+                        dev_status, stream):
+    if len(Ts) != len(Ms):
+        raise ValueError("one M per matrix")
+    x1 = x.reshape(-1)
+    if x1.numel() != K:
+        raise ValueError(f"x has {x1.numel()} values, expected K={K}")
+    if x1.dtype not in _DTYPE_CODE or y_dtype not in _DTYPE_CODE:
+        raise TypeError("activations and outputs must be float32, float16 or bfloat16")
+    if outs is None:
+        outs = [torch.empty((1, int(M)), dtype=y_dtype, device=x1.device) for M in Ms]
+    if len(outs) != len(Ts) or any(o.dtype != outs[0].dtype for o in outs):
+        raise ValueError("one output per matrix, all of one dtype")
+    descs = (GemvDesc * len(Ts))(*[GemvDesc(_ptr(T), int(M), _ptr(o))
+                                   for T, M, o in zip(Ts, Ms, outs)])
+    ytype = _DTYPE_CODE[outs[0].dtype] if outs else _DTYPE_CODE[y_dtype]
+    _check(getattr(lib, name)(ctypes.cast(descs, ctypes.c_void_p), len(Ts), int(K), _ptr(x1),
+                              _DTYPE_CODE[x1.dtype], ytype, int(flags), _ptr(dev_status),
+                              _stream(stream)), name)
+    return outs
+
+
+def gq_gemv_q4_0_tiled_grouped(Ts, Ms, K: int, x: torch.Tensor, y_dtype=torch.float16,
+                               outs=None, flags: int = 0, dev_status: torch.Tensor | None = None,
+                               stream=None):
+    """[y_i = W_hat_i @ x for each Q4_0 matrix in tiled storage T_i (M_i x K)], one fp16 x."""
+    return _gemv_tiled_grouped("gq_gemv_q4_0_tiled_grouped", Ts, Ms, K, x, y_dtype, outs, flags,
+                               dev_status, stream)
+
+
+def gq_gemv_ksb_tiled_grouped(Ts, Ms, K: int, x: torch.Tensor, y_dtype=torch.float16,
+                              outs=None, flags: int = 0, dev_status: torch.Tensor | None = None,
+                              stream=None):
+    """[y_i = W_hat_i @ x for each super-block matrix in tiled storage T_i], one fp16 x."""
+    return _gemv_tiled_grouped("gq_gemv_ksb_tiled_grouped", Ts, Ms, K, x, y_dtype, outs, flags,
+                               dev_status, stream)

@@ -66,6 +66,7 @@ constexpr int kRows = 16;
 constexpr int kCons = GQ_TILED_CONS;           // consumer warps (warps 1..kCons)
 constexpr int kThreads = 32 * (1 + kCons);
 constexpr int kRing = 4;                       // shared-memory stages
+static_assert((kRing & (kRing - 1)) == 0, "ring slots are taken as j & (kRing - 1)");
 constexpr int kStageBytes = 18432;             // a full Q4_0 tile; a ksb tile is 17664
 constexpr int kStageWords = 160 / kCons;       // words per lane, warp and stage (10 or 20)
 constexpr int kWordsA = kStageWords >= 16 ? 16 : 8;   // stash words of a stage in column block A
@@ -121,6 +122,43 @@ struct TArgs {
   int tgroups;  // row groups the partial-sum table holds
   uint32_t xf_off, xc_off, tab_off, bar_off;  // shared-memory layout
 };
+
+// Several matrices in one launch (they share K and x): their 16-row groups
+// are numbered one after the other, matrix i owning groups [gend[i-1],
+// gend[i]).  Passed by value, read from the kernel parameter space.
+constexpr int kMaxTiledMats = 256;
+struct TiledMat {
+  const uint8_t* T;
+  void* y;
+  int64_t M;
+  int gend;
+  int pad;
+};
+struct TiledTable {
+  TiledMat m[kMaxTiledMats];
+};
+struct OneMatrix {  // the single-matrix form: everything is in TArgs
+  int unused;
+};
+
+// Where row group g lives: its tiles, its outputs, and its group within its
+// matrix.  Each caller visits groups in increasing order, so the cursor mi
+// only moves forward.
+struct GroupAt {
+  const uint8_t* T;
+  void* y;
+  int64_t M, lg;
+};
+template <class Tbl>
+__device__ __forceinline__ GroupAt group_at(const TArgs& a, const Tbl& tbl, int64_t g, int& mi) {
+  if constexpr (sizeof(Tbl) == sizeof(OneMatrix)) {
+    return GroupAt{a.T, a.y, a.M, g};
+  } else {
+    while (g >= tbl.m[mi].gend) ++mi;
+    const int gb = mi ? tbl.m[mi - 1].gend : 0;
+    return GroupAt{tbl.m[mi].T, tbl.m[mi].y, tbl.m[mi].M, g - gb};
+  }
+}
 
 extern __shared__ __align__(1024) uint8_t smem[];
 
@@ -351,8 +389,8 @@ __device__ __forceinline__ void mbar_arrive_n(uint64_t* bar, uint32_t n) {
                : "memory");
 }
 
-template <int FMT>
-__global__ void __launch_bounds__(kThreads, 2) gemv_tiled_kernel(const TArgs a) {
+template <int FMT, class Tbl>
+__global__ void __launch_bounds__(kThreads, 2) gemv_tiled_kernel(const TArgs a, const Tbl tbl) {
   using F = Tile<FMT>;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + a.bar_off);
   uint64_t* empty = full + kRing;
@@ -400,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tiled_kernel(const TArgs a) 
       const uint64_t pol = policy_evict_first();
       int issued = 0;
       bool ok = true;
-      int s = 0;
+      int s = 0, pmi = 0;
       uint32_t ph = 0;
       for (int j = 0; j < ns; ++j) {
         if (!mbar_wait(&empty[s], ph ^ 1u, a.budget)) {
@@ -410,11 +448,12 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tiled_kernel(const TArgs a) 
         int64_t g;
         int c;
         stage_tile(j, g, c);
+        const GroupAt at = group_at(a, tbl, g, pmi);
         const int nb = (c == a.ntiles - 1) ? last_nb : F::kPerTile;
         const uint32_t bytes = static_cast<uint32_t>(nb * kRows * F::kBlkB);
         mbar_arrive_expect_tx(&full[s], bytes);
         bulk_g2s(smem + s * kStageBytes,
-                 a.T + g * a.group_bytes + static_cast<int64_t>(c) * F::kTileBytes, bytes,
+                 at.T + at.lg * a.group_bytes + static_cast<int64_t>(c) * F::kTileBytes, bytes,
                  &full[s], pol);
         ++issued;
         if (++s == kRing) {
@@ -545,12 +584,14 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tiled_kernel(const TArgs a) 
   };
   // the sum of slot `slot` over the warps (lanes 0..15: one row each): the
   // output of row group g
+  int fmi = 0;
   auto finish = [&](int slot, int64_t g) {
     float v = 0.f;
 #pragma unroll
     for (int ww = 0; ww < kCons; ++ww) v += tab[(slot * kCons + ww) * kRows + lane];
-    const int64_t row = g * kRows + lane;
-    if (row < a.M) store_elem(a.y, row, v * 16777216.0f, a.ytype);  // * 2^24
+    const GroupAt at = group_at(a, tbl, g, fmi);
+    const int64_t row = at.lg * kRows + lane;
+    if (row < at.M) store_elem(at.y, row, v * 16777216.0f, a.ytype);  // * 2^24
   };
 
   int j = 0;
@@ -667,9 +708,10 @@ size_t tiled_smem(int K, int& tgroups, uint32_t& xf, uint32_t& xc, uint32_t& tab
   return bar + kBarBytes;
 }
 
-template <int FMT>
-gq_status launch_tiled(const TArgs& a0, int grid, size_t smem_bytes, bool pdl, cudaStream_t stream) {
-  auto kern = gemv_tiled_kernel<FMT>;
+template <int FMT, class Tbl>
+gq_status launch_tiled(const TArgs& a0, const Tbl& tbl, int grid, size_t smem_bytes, bool pdl,
+                       cudaStream_t stream) {
+  auto kern = gemv_tiled_kernel<FMT, Tbl>;
   thread_local unsigned long long configured_ctx = 0;  // per host thread and context
   const unsigned long long ctx = context_id();
   if (ctx == 0 || ctx != configured_ctx) {
@@ -681,7 +723,7 @@ gq_status launch_tiled(const TArgs& a0, int grid, size_t smem_bytes, bool pdl, c
       return GQ_ERR_CUDA;
     configured_ctx = ctx;
   }
-  return launch(kern, dim3(grid), dim3(kThreads), smem_bytes, stream, pdl, a0);
+  return launch(kern, dim3(grid), dim3(kThreads), smem_bytes, stream, pdl, a0, tbl);
 }
 
 template <int FMT>
@@ -724,7 +766,81 @@ gq_status gemv_tiled_entry(const void* T, int64_t M, int64_t K, const void* x, i
   // waits, and only when the ring alone cannot hold the CTA's share
   a.stash = (pdl && stages > kRing) ? kStashMax : 0;
   const size_t smem_bytes = tiled_smem(a.K, a.tgroups, a.xf_off, a.xc_off, a.tab_off, a.bar_off);
-  return launch_tiled<FMT>(a, grid, smem_bytes, pdl, s);
+  return launch_tiled<FMT>(a, OneMatrix{}, grid, smem_bytes, pdl, s);
+}
+
+// Several tiled matrices that share K and x: y_i = W_i x for each descriptor
+// (W_i in tiled storage), in launches of up to kMaxTiledMats matrices whose
+// CTAs stream the row groups of all of them back to back.
+template <int FMT>
+gq_status gemv_tiled_grouped_entry(const gq_gemv_desc* mats, int count, int64_t K,
+                                   const void* x, int x_dtype, int y_dtype, unsigned flags,
+                                   int* dev_status, void* stream) {
+  if (count < 0 || K < 0) return GQ_ERR_INVALID_ARG;
+  if (count > 0 && !mats) return GQ_ERR_INVALID_ARG;
+  if (x_dtype != GQ_F16 || !valid_act_dtype(y_dtype)) return GQ_ERR_DTYPE;
+  if (flags & ~GQ_GEMV_PDL) return GQ_ERR_INVALID_ARG;
+  if (!unit_shape(FMT, K) || K > kMaxKb * 32) return GQ_ERR_SHAPE;
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return GQ_ERR_ALIGNMENT;
+  int64_t groups = 0;
+  for (int i = 0; i < count; ++i) {
+    const gq_gemv_desc& d = mats[i];
+    if (d.M < 0) return GQ_ERR_INVALID_ARG;
+    if (d.M > 0x7FFFFFFFLL) return GQ_ERR_SHAPE;
+    if (d.M == 0) continue;
+    if (!d.y || (K > 0 && !d.W)) return GQ_ERR_INVALID_ARG;
+    if (misaligned16(d.y) || misaligned16(d.W)) return GQ_ERR_ALIGNMENT;
+    groups += (d.M + kRows - 1) / kRows;
+  }
+  if (groups > 0x7FFFFFFFLL) return GQ_ERR_SHAPE;
+  if (groups == 0) return GQ_OK;
+  cudaStream_t s = as_stream(stream);
+  if (K == 0) {
+    for (int i = 0; i < count; ++i)
+      if (mats[i].M > 0 &&
+          cudaMemsetAsync(mats[i].y, 0, static_cast<size_t>(mats[i].M * dtype_size(y_dtype)), s) !=
+              cudaSuccess)
+        return GQ_ERR_CUDA;
+    return GQ_OK;
+  }
+  if (!x) return GQ_ERR_INVALID_ARG;
+  if (misaligned16(x)) return GQ_ERR_ALIGNMENT;
+  const bool pdl = (flags & GQ_GEMV_PDL) != 0;
+
+  TArgs a{};
+  a.x = static_cast<const __half*>(x);
+  a.dev_status = dev_status;
+  a.budget = kWaitBudget;
+  a.group_bytes = kRows * canon_row_bytes(FMT, K);
+  a.K = static_cast<int>(K);
+  a.ytype = y_dtype;
+  a.nblk = static_cast<int>(FMT == GQ_FMT_Q4_0 ? K / 32 : K / 256);
+  a.ntiles = (a.nblk + Tile<FMT>::kPerTile - 1) / Tile<FMT>::kPerTile;
+  const size_t smem_bytes = tiled_smem(a.K, a.tgroups, a.xf_off, a.xc_off, a.tab_off, a.bar_off);
+  TiledTable tbl{};  // one launch's table, passed to the kernel by value
+  int i = 0;
+  while (i < count) {
+    int n = 0, g = 0;
+    for (; i < count && n < kMaxTiledMats; ++i) {
+      const gq_gemv_desc& d = mats[i];
+      if (d.M == 0) continue;
+      g += static_cast<int>((d.M + kRows - 1) / kRows);
+      tbl.m[n] = TiledMat{static_cast<const uint8_t*>(d.W), d.y, d.M, g, 0};
+      ++n;
+    }
+    if (n == 0) break;
+    a.ngroups = g;
+    // Two CTAs per SM from this one launch, each taking its first stages
+    // through tensor memory whether or not the launch overlaps another: on
+    // long grouped streams this measured faster than one CTA per SM (with or
+    // without the stash) and than two CTAs per SM without it.
+    const int grid = g < 2 * sm_count() ? g : 2 * sm_count();
+    const int64_t stages = ((static_cast<int64_t>(g) + grid - 1) / grid) * a.ntiles;
+    a.stash = stages > kRing ? kStashMax : 0;
+    const gq_status st = launch_tiled<FMT>(a, tbl, grid, smem_bytes, pdl, s);
+    if (st != GQ_OK) return st;
+  }
+  return GQ_OK;
 }
 
 template <int FMT>
@@ -775,6 +891,20 @@ GQ_API gq_status gq_gemv_ksb_tiled(const void* T, int64_t M, int64_t K, const vo
                                    void* stream) {
   return gq::gemv_tiled_entry<GQ_FMT_KSB>(T, M, K, x, x_dtype, y, y_dtype, flags, dev_status,
                                           stream);
+}
+
+GQ_API gq_status gq_gemv_q4_0_tiled_grouped(const gq_gemv_desc* mats, int count, int64_t K,
+                                            const void* x, int x_dtype, int y_dtype,
+                                            unsigned flags, int* dev_status, void* stream) {
+  return gq::gemv_tiled_grouped_entry<GQ_FMT_Q4_0>(mats, count, K, x, x_dtype, y_dtype, flags,
+                                                   dev_status, stream);
+}
+
+GQ_API gq_status gq_gemv_ksb_tiled_grouped(const gq_gemv_desc* mats, int count, int64_t K,
+                                           const void* x, int x_dtype, int y_dtype,
+                                           unsigned flags, int* dev_status, void* stream) {
+  return gq::gemv_tiled_grouped_entry<GQ_FMT_KSB>(mats, count, K, x, x_dtype, y_dtype, flags,
+                                                  dev_status, stream);
 }
 
 }  // extern "C"

@@ -268,6 +268,26 @@ GQ_API gq_status gq_gemv_ksb_tiled(const void* T, int64_t M, int64_t K, const vo
                                    void* y, int y_dtype, unsigned flags, int* dev_status,
                                    void* stream);
 
+/* Grouped tiled GEMV (no counterpart on the pages: the GGUF GEMV of the format
+ * pages applied to many tiled matrices that share one activation vector, e.g.
+ * every projection of a decoder layer or of a whole model in one call).
+ * y_i = W_i x for each descriptor, each output as gq_gemv_*_tiled computes it
+ * (the same fp32 additions in the same order, so bit for bit the same).
+ *   mats:  count host descriptors {W, M, y} (read during the call only); W is
+ *          the TILED storage of an M x K matrix (gq_repack_*), y: [M] of
+ *          y_dtype; both 16-byte aligned.  M == 0 entries are skipped (W and
+ *          y may then be NULL).
+ *   K, x, x_dtype, y_dtype, flags, dev_status: as for gq_gemv_*_tiled, shared
+ *          by all matrices (B = 1, fp16 x).
+ * Validation covers every descriptor before anything is launched; more than
+ * 256 matrices are processed in several launches in stream order. */
+GQ_API gq_status gq_gemv_q4_0_tiled_grouped(const gq_gemv_desc* mats, int count, int64_t K,
+                                            const void* x, int x_dtype, int y_dtype,
+                                            unsigned flags, int* dev_status, void* stream);
+GQ_API gq_status gq_gemv_ksb_tiled_grouped(const gq_gemv_desc* mats, int count, int64_t K,
+                                           const void* x, int x_dtype, int y_dtype,
+                                           unsigned flags, int* dev_status, void* stream);
+
 /* Allocation-free variant (no counterpart on the pages): the batch-1 integer
  * tensor-core path of gq_gemv_q4_0 (fp16 x, B = 1) with its scratch -- the
  * per-CTA counts and partial sums, 33 KB -- in a static device array of the

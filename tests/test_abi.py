@@ -152,6 +152,35 @@ def test_gemv_grouped_validation():
         assert call([good], B=0) == GQ_OK
 
 
+def test_gemv_tiled_grouped_validation():
+    import ctypes
+    D = gq.GemvDesc
+    for name, K in (("gq_gemv_q4_0_tiled_grouped", 64), ("gq_gemv_ksb_tiled_grouped", 256)):
+        f = getattr(gq.lib, name)
+
+        def call(descs, count=None, K=K, x=A, xt=gq.GQ_F16, yt=gq.GQ_F16, flags=0, st=None):
+            arr = (D * max(len(descs), 1))(*descs)
+            n = len(descs) if count is None else count
+            return f(ctypes.cast(arr, ctypes.c_void_p), n, K, x, xt, yt, flags, st, None)
+
+        good = D(A, 16, A + 4096)
+        assert call([good], count=-1) == INVALID
+        assert f(None, 1, K, A, gq.GQ_F16, gq.GQ_F16, 0, None, None) == INVALID
+        assert call([D(A, -1, A)]) == INVALID
+        assert call([good, D(A + 2, 16, A)]) == ALIGN           # every descriptor is checked
+        assert call([good, D(A, 16, A + 8)]) == ALIGN
+        assert call([good, D(None, 16, A)]) == INVALID
+        assert call([good, D(A, 16, None)]) == INVALID
+        assert call([good], K=K + 32) == SHAPE                 # not whole tiles of units
+        assert call([good], K=16384 + 256) == SHAPE
+        assert call([good], xt=gq.GQ_BF16) == DTYPE and call([good], yt=7) == DTYPE
+        assert call([good], flags=2) == INVALID
+        assert call([good], x=None) == INVALID and call([good], x=A + 2) == ALIGN
+        assert call([good], st=A + 2) == ALIGN
+        assert call([], count=0) == GQ_OK                      # nothing to do: no launch
+        assert call([D(None, 0, None), D(None, 0, None)]) == GQ_OK
+
+
 def test_binding_refuses_host_tensors():
     import torch
     with pytest.raises(ValueError):

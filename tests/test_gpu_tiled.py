@@ -171,3 +171,108 @@ def test_tiled_gemv_nonfinite_activation(fmt, bad):
     for flags in (0, gq.GQ_GEMV_PDL):
         y = run(fmt, T, M, K, x, torch.float32, flags)
         assert not bool(torch.isfinite(y).any())
+
+
+def grouped(fmt):
+    return gq.gq_gemv_q4_0_tiled_grouped if fmt == Q40 else gq.gq_gemv_ksb_tiled_grouped
+
+
+@pytest.mark.parametrize("fmt", [Q40, KSB])
+def test_tiled_grouped_decoder_layer(fmt):
+    # the seven projections of one decoder layer of the 4096 / 11008 model
+    # that share one input (four 4096-row, three 11008-row matrices, K = 4096)
+    # in one call; each output is bit for bit the single-matrix tiled GEMV's
+    K = 4096
+    Ms = [4096] * 4 + [11008] * 3
+    qs = [packed(fmt, M, K, seed=100 + i) for i, M in enumerate(Ms)]
+    Ts = [tiled(fmt, q, M, K) for q, M in zip(qs, Ms)]
+    x = synth.activations(1, K, seed=21, dtype=torch.float16)
+    xd = x.cuda()
+    for flags in (0, gq.GQ_GEMV_PDL):
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        ys = grouped(fmt)(Ts, Ms, K, xd, y_dtype=torch.float32, flags=flags, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        for q, T, M, y in zip(qs, Ts, Ms, ys):
+            Y, bound = oracle.gemm(fmt, q, M, K, *x_for_oracle(x))
+            assert_product_close(y, Y, bound)
+            assert torch.equal(y, run(fmt, T, M, K, x, torch.float32, flags))
+
+
+@pytest.mark.parametrize("fmt,K", [(Q40, 1088), (KSB, 2304), (Q40, 16384), (KSB, 16384)])
+def test_tiled_grouped_ragged(fmt, K):
+    # ragged row counts (one row, a partial group, exact groups), an empty
+    # entry in the middle, and bfloat16 outputs
+    Ms = [1, 17, 0, 48, 333, 16]
+    qs = [packed(fmt, M, K, seed=7 * i + K) if M else None for i, M in enumerate(Ms)]
+    Ts = [tiled(fmt, q, M, K) if M else torch.empty(0, dtype=torch.uint8, device="cuda")
+          for q, M in zip(qs, Ms)]
+    x = synth.activations(1, K, seed=K + 3, dtype=torch.float16)
+    for flags in (0, gq.GQ_GEMV_PDL):
+        ys = grouped(fmt)(Ts, Ms, K, x.cuda(), y_dtype=torch.bfloat16, flags=flags)
+        torch.cuda.synchronize()
+        for q, M, y in zip(qs, Ms, ys):
+            if M == 0:
+                assert y.numel() == 0
+                continue
+            Y, bound = oracle.gemm(fmt, q, M, K, *x_for_oracle(x))
+            assert_product_close(y, Y, bound)
+
+
+@pytest.mark.parametrize("fmt", [Q40, KSB])
+def test_tiled_grouped_more_than_one_launch(fmt):
+    # 300 matrices: more than one launch's table of 256, in stream order
+    K = 1024 if fmt == Q40 else 2048
+    Ms = [16 + (i % 5) * 7 for i in range(300)]
+    q = packed(fmt, max(Ms), K, seed=9)
+    rb = len(q) // max(Ms)
+    T_by_M = {M: tiled(fmt, q[:M * rb], M, K) for M in set(Ms)}
+    x = synth.activations(1, K, seed=2, dtype=torch.float16)
+    ys = grouped(fmt)([T_by_M[M] for M in Ms], Ms, K, x.cuda(), y_dtype=torch.float32,
+                      flags=gq.GQ_GEMV_PDL)
+    torch.cuda.synchronize()
+    want = {M: oracle.gemm(fmt, q[:M * rb], M, K, *x_for_oracle(x)) for M in set(Ms)}
+    for M, y in zip(Ms, ys):
+        assert_product_close(y, *want[M])
+
+
+@pytest.mark.parametrize("fmt", [Q40, KSB])
+def test_tiled_grouped_stays_in_bounds(fmt):
+    # every output of the table gets exactly its M values: sentinel bytes
+    # around each output stay untouched
+    K = 2048
+    Ms = [33, 16, 70]
+    guard, sent = 256, 0xA5
+    qs = [packed(fmt, M, K, seed=40 + M) for M in Ms]
+    Ts = [tiled(fmt, q, M, K) for q, M in zip(qs, Ms)]
+    bufs = [torch.full((4 * M + 2 * guard,), sent, dtype=torch.uint8, device="cuda") for M in Ms]
+    outs = [b[guard:guard + 4 * M].view(torch.float32).view(1, M) for b, M in zip(bufs, Ms)]
+    x = synth.activations(1, K, seed=8, dtype=torch.float16)
+    grouped(fmt)(Ts, Ms, K, x.cuda(), outs=outs, flags=gq.GQ_GEMV_PDL)
+    torch.cuda.synchronize()
+    for b in bufs:
+        assert bool((b[:guard] == sent).all()) and bool((b[-guard:] == sent).all())
+    for q, M, y in zip(qs, Ms, outs):
+        assert_product_close(y, *oracle.gemm(fmt, q, M, K, *x_for_oracle(x)))
+
+
+
+@pytest.mark.parametrize("fmt", [Q40, KSB])
+def test_tiled_grouped_table_batches(fmt):
+    # K = 16384 leaves room for six row groups in the partial-sum table;
+    # two 16576-row matrices are 2072 row groups, seven per CTA on two CTAs
+    # per SM of 148 SMs: the table is filled, reduced and filled again.  The
+    # same weights twice, so both outputs must match the oracle and each other.
+    M, K = 16576, 16384
+    q = packed(fmt, M, K)
+    T = tiled(fmt, q, M, K)
+    x = synth.activations(1, K, seed=6, dtype=torch.float16)
+    Y, bound = oracle.gemm(fmt, q, M, K, *x_for_oracle(x))
+    for flags in (0, gq.GQ_GEMV_PDL):
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        ys = grouped(fmt)([T, T], [M, M], K, x.cuda(), y_dtype=torch.float32, flags=flags,
+                          dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        assert_product_close(ys[0], Y, bound)
+        assert torch.equal(ys[0], ys[1])
