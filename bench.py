@@ -471,6 +471,44 @@ def extra_rows(gq, synth, dev, peak, bf16):
                                  "weight_gbs": round(nb / (ms * 1e-3) / 1e9, 1)}
         del Wc
     out["batch8"] = dict(workload="W 11008x4096, X fp16 [8, 4096], Y fp16, 6 rotated copies", **b8)
+
+    # small batches on the transposed shape, where x of 6..16 rows no longer
+    # fits beside the weight ring: K split over clusters of 2..3 CTAs
+    M, K = 4096, 11008
+    bk = {}
+    for fmt in ("q4_0", "ksb"):
+        w = synth.gaussian_weights(M, K, seed=13, device=dev) if fmt == "q4_0" else \
+            synth.logstd_weights(M, K, seed=3, device=dev)
+        q = quant(fmt, w)
+        del w
+        nb = q.numel()
+        copies = 6
+        Wc = torch.empty((copies, nb), dtype=torch.uint8, device=dev)
+        Wc.copy_(q.view(1, nb).expand(copies, nb))
+        f = gq.gq_gemv_q4_0 if fmt == "q4_0" else gq.gq_gemv_ksb
+        fm = gq.gq_gemm_q4_0 if fmt == "q4_0" else gq.gq_gemm_ksb
+        bk[fmt] = {}
+        for B in (2, 4, 8, 16):
+            if B <= 8:
+                xb = synth.activations(B, K, seed=B, dtype=torch.float16, device=dev)
+                yb = torch.empty((B, M), dtype=torch.float16, device=dev)
+                ms = _graph_ms(lambda: [f(Wc[i], M, K, xb, out=yb, flags=gq.GQ_GEMV_PDL)
+                                        for i in range(copies)], 20) / copies
+            else:
+                xb = synth.activations(B, K, seed=B, dtype=torch.bfloat16, device=dev)
+                yb = torch.empty((B, M), dtype=torch.float32, device=dev)
+                wsp = torch.zeros(max(gq.gq_gemm_workspace_bytes(
+                    gq.GQ_FMT_Q4_0 if fmt == "q4_0" else gq.GQ_FMT_KSB, M, K, B), 1),
+                    dtype=torch.uint8, device=dev)
+                ms = _graph_ms(lambda: [fm(Wc[i], M, K, xb, out=yb, workspace=wsp)
+                                        for i in range(copies)], 20) / copies
+            gbs = nb / (ms * 1e-3) / 1e9
+            bk[fmt][str(B)] = {"us": round(ms * 1e3, 3), "gbs": round(gbs, 1),
+                               "frac_of_peak": frac(gbs)}
+        del Wc
+    out["batches_4096x11008"] = dict(
+        workload="W 4096x11008, X [B, 11008] (fp16 through gq_gemv_* for B <= 8 with PDL, bf16 "
+                 "through gq_gemm_* for B = 16), 6 rotated copies", **bk)
     out["gemm"] = dict(workload="W 11008x4096, X bf16 [B, 4096], Y fp32, 6 rotated copies; "
                                 "useful flops 2*M*K*B", **gemm)
 

@@ -83,6 +83,8 @@ constexpr int kMaxNT = 2;
 // cross-warp reduction buffer of a launch with NT tiles (two groups in flight)
 constexpr int red_bytes(int nt) { return 2 * kConsumers * 32 * acc_len(nt) * 4; }
 constexpr int kRedBytes = red_bytes(kMaxNT);  // the largest
+// exchange slots of a cluster's K split (groups one rank may run ahead)
+constexpr int kSplitSlots = 4;
 // activation window budget: what the stages and the reduction leave of the
 // 227 KB a CTA may hold, at most 72 KB
 constexpr int kXSmemFree = 227 * 1024 - kStages * kStageBytes - kRedBytes - 1024;
@@ -92,6 +94,15 @@ static_assert(kChunkW == 1024 || kChunkW == 2048, "supported chunk sizes");
 static_assert(kSubPerWarp % 2 == 0, "blocks per warp come in pairs");
 
 enum { XT_F16 = 0, XT_BF16 = 1, XT_F32 = 2 };
+
+// Smallest batch that keeps all of x resident beyond the window budget.  The
+// large-table configuration keeps its windows so that its small CTAs stay
+// several per SM.
+#if GQ_GEMV_MANY_TU
+constexpr int kResidentMinB = 9;
+#else
+constexpr int kResidentMinB = 2;
+#endif
 
 
 template <int FMT>
@@ -114,6 +125,10 @@ struct GemvArgs {
   long long budget;
   int B, ytype, nchunks, win, ngroups;  // win: chunks per activation window
   int skip_first;  // self-test only: never fill the first stage, so waits run out
+  // K split over a cluster: chunks per CTA, and the shared-memory offset of
+  // the exchange area (barriers, then the partial sums)
+  int split_cps;
+  uint32_t split_off;
 };
 
 // Matrices of one launch.  A single product reads W, M and y from GemvArgs
@@ -523,8 +538,13 @@ __device__ void load_x_window(uint8_t* xs, const void* x, int64_t K, int B, int 
   }
 }
 
-template <int FMT, int XT, int NT, bool ALIGNED, class Tbl>
-__global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
+// SPLIT: the CTAs of a cluster share each row group, CTA rank q taking the
+// chunks [q * split_cps, (q + 1) * split_cps) of every row with its slice of
+// x resident; rank 0 adds the other ranks' partial sums, in rank order, read
+// from their shared memory, and stores y.  A slice of x fills more than half
+// of the shared memory, so these CTAs run one per SM.
+template <int FMT, int XT, int NT, bool ALIGNED, class Tbl, bool SPLIT = false>
+__global__ void __launch_bounds__(kThreads, SPLIT ? 1 : GQ_GEMV_MINB)
     gemv_kernel(const GemvArgs a, const __grid_constant__ Tbl tbl) {
   constexpr int kBlkW = Fmt<FMT>::kBlkW, kBlkB = Fmt<FMT>::kBlkB;
   constexpr int kTerms = (XT == XT_F32) ? 3 : 1;
@@ -540,10 +560,29 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
   uint64_t* empty = full + kStages;
   uint64_t* cbar = empty + kStages;  // consumer-group barrier (bounded waits)
   int* abort_flag = reinterpret_cast<int*>(cbar + 1);
+  // SPLIT exchange: every rank leaves its partial sums of group gi in its
+  // xred slot gi % kSplitSlots; part_full[p] (rank 0) completes when every
+  // lane of every other rank has done so, part_free[p] (other ranks) when
+  // rank 0's lanes have read them.  Rank 0 adds up a group one group later,
+  // so that its wait rarely holds up its own pipeline.
+  uint64_t* part_full = reinterpret_cast<uint64_t*>(smem + a.split_off);
+  uint64_t* part_free = part_full + kSplitSlots;
+  float* xred = reinterpret_cast<float*>(part_free + kSplitSlots);  // [slots][32][acc_len(NT)]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nblk_row = static_cast<int>(a.K / kBlkW);
   const int nfull = nblk_row / kBlkPerChunk;  // chunks with every block present
+  // this CTA's chunks of a row and its row groups g_first, g_first + g_step, ...
+  int c_begin = 0, c_end = a.nchunks, g_first = blockIdx.x, g_step = gridDim.x;
+  uint32_t rank = 0, nrank = 1;
+  if constexpr (SPLIT) {
+    rank = cluster_ctarank();
+    nrank = cluster_nctarank();
+    c_begin = static_cast<int>(rank) * a.split_cps;
+    c_end = min(a.nchunks, c_begin + a.split_cps);
+    g_first = static_cast<int>(cluster_id_x());
+    g_step = static_cast<int>(cluster_count_x());
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -551,10 +590,18 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
       mbar_init(&empty[s], kConsumers);
     }
     mbar_init(cbar, kConsumers);
+    if constexpr (SPLIT) {
+      for (int p = 0; p < kSplitSlots; ++p) {
+        mbar_init(&part_full[p], 32 * (nrank - 1));
+        mbar_init(&part_free[p], 32);
+      }
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
   __syncthreads();
+  // every CTA's barriers exist before any other CTA of the cluster arrives on them
+  if constexpr (SPLIT) cluster_sync_all();
   pdl_launch_dependents();
 
   if (warp == 0) {
@@ -566,13 +613,14 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
     bool ok = true;
     const uint32_t tail_bytes = static_cast<uint32_t>((nblk_row - nfull * kBlkPerChunk) * kBlkB);
     int pmi = 0;  // matrix cursor
-    for (int g = blockIdx.x; g < a.ngroups && ok; g += gridDim.x) {
+    for (int g = g_first; g < a.ngroups && ok; g += g_step) {
       const Unit un = unit_of(a, tbl, g, pmi);
       const int64_t m0 = un.m0;
       const bool row_ok = lane < kRows && m0 + lane < un.M;
       uintptr_t src = reinterpret_cast<uintptr_t>(un.W) +
-                      static_cast<uintptr_t>((m0 + (row_ok ? lane : 0)) * a.rowbytes);
-      for (int c = 0; c < a.nchunks; ++c, ++issued, src += kChunkBytes) {
+                      static_cast<uintptr_t>((m0 + (row_ok ? lane : 0)) * a.rowbytes +
+                                             static_cast<int64_t>(c_begin) * kChunkBytes);
+      for (int c = c_begin; c < c_end; ++c, ++issued, src += kChunkBytes) {
         if (!mbar_wait(&empty[s], ph ^ 1u, a.budget) ||
             *reinterpret_cast<volatile int*>(abort_flag)) {
           ok = false;
@@ -621,6 +669,8 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
         }
       }
     }
+    // no CTA of the cluster leaves while another may still read its memory
+    if constexpr (SPLIT) cluster_sync_all();
     return;
   }
 
@@ -650,9 +700,9 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
 
   pdl_wait();  // the preceding grid has finished: x is ready, y may be written
 
-  const bool x_resident = (a.win >= a.nchunks);
+  const bool x_resident = (a.win >= c_end - c_begin);
   if (x_resident) {
-    load_x_window<XT>(xs, a.x, a.K, a.B, 0, a.win, term_stride, ctid);
+    load_x_window<XT>(xs, a.x, a.K, a.B, c_begin, a.win, term_stride, ctid);
     ok = group_sync();
   }
   const uint32_t x_chunk = static_cast<uint32_t>(a.B * kXStride);
@@ -660,25 +710,86 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
   // n8 tile 1 holds batch rows 8..15: this lane's row there, relative to tile 0
   const uint32_t xt1 = static_cast<uint32_t>((min(8 + r, a.B - 1) - bsel) * kXStride);
 
+  constexpr int kTiles = NT > 1 ? NT : 1;
+  // y at rows m0 + r and m0 + r + 8 of the batch columns this lane holds
+  // (NT = 0: lane t = 0 holds row r, lane t = 1 row r + 8, see scale_acc)
+  auto store_rows = [&](const float* v, void* y, int64_t M, int64_t m0) {
+    const int64_t ra = m0 + r, rbw = m0 + r + 8;
+    if constexpr (NT == 0) {
+      const int64_t row = (t == 0) ? ra : rbw;
+      if (t < 2 && row < M) store_elem(y, row, v[0], a.ytype);
+    } else {
+#pragma unroll
+      for (int n = 0; n < kTiles; ++n) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int col = 8 * n + 2 * t + i;
+          if (col < a.B) {
+            if (ra < M) store_elem(y, col * M + ra, v[4 * n + i], a.ytype);
+            if (rbw < M) store_elem(y, col * M + rbw, v[4 * n + 2 + i], a.ytype);
+          }
+        }
+      }
+    }
+  };
+  // SPLIT, rank 0, warp 0: add up group gj (row group gg) from every rank's
+  // slot, in rank order, and store it.  Each lane reads and releases only
+  // its own entries.
+  auto split_finish = [&](int gj, int gg) -> bool {
+    const int p = gj % kSplitSlots;
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait_cluster(&part_full[p],
+                                                   static_cast<uint32_t>(gj / kSplitSlots) & 1u,
+                                                   a.budget)))
+      return false;
+    const float4* slot = reinterpret_cast<const float4*>(xred) + (p * 32 + lane) * kTiles;
+    float v[acc_len(NT)];
+#pragma unroll
+    for (int n = 0; n < kTiles; ++n) {
+      const float4 o = slot[n];
+      v[4 * n + 0] = o.x;
+      v[4 * n + 1] = o.y;
+      v[4 * n + 2] = o.z;
+      v[4 * n + 3] = o.w;
+    }
+    const uint32_t sa = smem_addr(slot);
+    for (uint32_t q = 1; q < nrank; ++q) {
+#pragma unroll
+      for (int n = 0; n < kTiles; ++n) {
+        const float4 w = ld_cluster_f4(sa + 16u * n, q);
+        v[4 * n + 0] += w.x;
+        v[4 * n + 1] += w.y;
+        v[4 * n + 2] += w.z;
+        v[4 * n + 3] += w.w;
+      }
+    }
+    for (uint32_t q = 1; q < nrank; ++q) mbar_arrive_remote(&part_free[p], q);
+    store_rows(v, a.y, a.M, static_cast<int64_t>(gg) * kRows);
+    return true;
+  };
+
   int s = 0;        // stage of the next use
   uint32_t ph = 0;  // its phase parity
   int gi = 0;       // groups done by this CTA
   int cmi = 0;  // matrix cursor
-  for (int g = blockIdx.x; g < a.ngroups && ok; g += gridDim.x, ++gi) {
+  for (int g = g_first; g < a.ngroups && ok; g += g_step, ++gi) {
     const Unit un = unit_of(a, tbl, g, cmi);
     const int64_t m0 = un.m0;
     float acc[acc_len(NT)];
 #pragma unroll
     for (int q = 0; q < acc_len(NT); ++q) acc[q] = 0.f;
-    // offset of row r's (and r+8's) first byte inside its 16-byte granule
+    // offset of row r's (and r+8's) first byte of chunk c_begin inside its
+    // 16-byte granule
+    const int64_t cb_off = static_cast<int64_t>(c_begin) * kChunkBytes;
     uint32_t off0 = static_cast<uint32_t>(
-        (reinterpret_cast<uintptr_t>(un.W) + static_cast<uintptr_t>((m0 + r) * a.rowbytes)) & 15u);
+        (reinterpret_cast<uintptr_t>(un.W) + static_cast<uintptr_t>((m0 + r) * a.rowbytes + cb_off)) &
+        15u);
     uint32_t off1 = static_cast<uint32_t>(
-        (reinterpret_cast<uintptr_t>(un.W) + static_cast<uintptr_t>((m0 + r + 8) * a.rowbytes)) &
+        (reinterpret_cast<uintptr_t>(un.W) +
+         static_cast<uintptr_t>((m0 + r + 8) * a.rowbytes + cb_off)) &
         15u);
     uint32_t xw = x_lane;
     int cw_in_win = 0;
-    for (int c = 0; c < a.nchunks; ++c) {
+    for (int c = c_begin; c < c_end; ++c) {
       if (!x_resident && cw_in_win == 0) {
         if (!group_sync()) { ok = false; break; }
         load_x_window<XT>(xs, a.x, a.K, a.B, c, a.win, term_stride, ctid);
@@ -729,7 +840,6 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
 
     // reduce the consumer warps' partial sums (double-buffered by group
     // parity, so one barrier per group suffices), then store
-    constexpr int kTiles = NT > 1 ? NT : 1;
     float4* rb = reinterpret_cast<float4*>(red) + (gi & 1) * kConsumers * 32 * kTiles;
 #pragma unroll
     for (int n = 0; n < kTiles; ++n)
@@ -751,31 +861,42 @@ __global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
           s4[4 * n + 3] += v.w;
         }
       }
-      const int64_t ra = m0 + r, rbw = m0 + r + 8;
-      if constexpr (NT == 0) {
-        // lane t = 0 holds row r, lane t = 1 row r + 8 (scale_acc)
-        const int64_t row = (t == 0) ? ra : rbw;
-        if (t < 2 && row < un.M) store_elem(un.y, row, s4[0], a.ytype);
-      } else {
+      if constexpr (SPLIT) {
+        const int p = gi % kSplitSlots;
+        float4* slot = reinterpret_cast<float4*>(xred) + (p * 32 + lane) * kTiles;
+        // rank 0 has read what this slot held kSplitSlots groups ago (its own
+        // slot it read itself, one group after writing it)
+        if (rank != 0 && gi >= kSplitSlots &&
+            !__all_sync(0xFFFFFFFFu,
+                        mbar_wait_cluster(&part_free[p],
+                                          static_cast<uint32_t>(gi / kSplitSlots - 1) & 1u,
+                                          a.budget))) {
+          ok = false;
+        } else {
 #pragma unroll
-        for (int n = 0; n < kTiles; ++n) {
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int col = 8 * n + 2 * t + i;
-            if (col < a.B) {
-              if (ra < un.M) store_elem(un.y, col * un.M + ra, s4[4 * n + i], a.ytype);
-              if (rbw < un.M) store_elem(un.y, col * un.M + rbw, s4[4 * n + 2 + i], a.ytype);
-            }
-          }
+          for (int n = 0; n < kTiles; ++n)
+            slot[n] = make_float4(s4[4 * n], s4[4 * n + 1], s4[4 * n + 2], s4[4 * n + 3]);
+          if (rank != 0) mbar_arrive_remote(&part_full[p], 0);
+          // the previous group's parts are in, or about to be
+          if (rank == 0 && gi >= 1 && !split_finish(gi - 1, g - g_step)) ok = false;
         }
+      } else {
+        store_rows(s4, un.y, un.M, m0);
       }
     }
+  }
+  // SPLIT: rank 0 adds up its last group
+  if constexpr (SPLIT) {
+    if (ok && cw == 0 && rank == 0 && gi >= 1 && !split_finish(gi - 1, g_first + (gi - 1) * g_step))
+      ok = false;
   }
 
   if (!ok && lane == 0) {
     report(a.dev_status, GQ_DEV_TIMEOUT);
     *reinterpret_cast<volatile int*>(abort_flag) = 1;
   }
+  // no CTA of the cluster leaves while another may still read its memory
+  if constexpr (SPLIT) cluster_sync_all();
 }
 
 size_t gemv_smem_bytes(int B, int terms, int win) {
@@ -822,6 +943,80 @@ gq_status launch_gemv(const GemvArgs& a, const Tbl& tbl, cudaStream_t stream, bo
   return launch(kern, dim3(grid), dim3(kThreads), smem, stream, pdl, a, tbl);
 }
 
+// Bytes of the K-split exchange area: kSplitSlots barriers each way, then
+// the partial sums [kSplitSlots][32][acc_len(nt)].
+constexpr size_t split_extra(int nt) {
+  return 16 * kSplitSlots + static_cast<size_t>(kSplitSlots) * 32 * acc_len(nt) * 4;
+}
+
+// One matrix with K split over clusters of `cluster` CTAs (a.split_cps chunks
+// each, a.win == a.split_cps).  Sets `launched` when it launched (or failed
+// to); leaves it false when no cluster of that size fits on the device.
+template <int FMT, int XT, int NT, bool ALIGNED>
+gq_status launch_gemv_split(GemvArgs a, int cluster, cudaStream_t stream, bool pdl,
+                            bool& launched) {
+  constexpr int kTerms = (XT == XT_F32) ? 3 : 1;
+  auto kern = gemv_kernel<FMT, XT, NT, ALIGNED, NoTable, true>;
+  const size_t base = (gemv_smem_bytes(a.B, kTerms, a.win) + 15) & ~static_cast<size_t>(15);
+  a.split_off = static_cast<uint32_t>(base);
+  const size_t smem = base + split_extra(NT);
+  // per host thread, as launch_gemv
+  thread_local unsigned long long configured_ctx = 0;
+  thread_local size_t configured_smem = 0;
+  thread_local size_t occ_smem = 0;
+  thread_local int occ_cluster = 0;
+  thread_local int max_clusters = 0;
+  const unsigned long long ctx = context_id();
+  launched = true;
+  if (ctx == 0 || ctx != configured_ctx || smem > configured_smem) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return GQ_ERR_CUDA;
+    configured_ctx = ctx;
+    configured_smem = smem;
+    occ_smem = 0;
+  }
+  if (occ_smem != smem || occ_cluster != cluster) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(cluster * sm_count()));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+      (void)cudaGetLastError();
+      n = 0;
+    }
+    max_clusters = n;
+    occ_smem = smem;
+    occ_cluster = cluster;
+  }
+  if (max_clusters < 1) {
+    launched = false;
+    return GQ_OK;
+  }
+  const int nclusters = a.ngroups < max_clusters ? a.ngroups : max_clusters;
+  return launch_cluster(kern, dim3(static_cast<unsigned>(nclusters * cluster)), dim3(kThreads),
+                        smem, stream, pdl, static_cast<unsigned>(cluster), a, NoTable{0});
+}
+
+template <int FMT, int XT>
+gq_status dispatch_split(const GemvArgs& a, int cluster, bool w_aligned, cudaStream_t s, bool pdl,
+                         bool& launched) {
+  const bool aligned = (a.rowbytes % 16 == 0) && w_aligned;
+  if (a.B <= 8)
+    return aligned ? launch_gemv_split<FMT, XT, 1, true>(a, cluster, s, pdl, launched)
+                   : launch_gemv_split<FMT, XT, 1, false>(a, cluster, s, pdl, launched);
+  return aligned ? launch_gemv_split<FMT, XT, 2, true>(a, cluster, s, pdl, launched)
+                 : launch_gemv_split<FMT, XT, 2, false>(a, cluster, s, pdl, launched);
+}
+
 // w_aligned: every matrix of the launch starts on a 16-byte boundary.
 template <int FMT, int XT, class Tbl>
 gq_status dispatch_gemv(const GemvArgs& a, const Tbl& tbl, bool w_aligned, cudaStream_t s,
@@ -865,12 +1060,15 @@ void fill_common(GemvArgs& a, int64_t K, const void* x, int xt, int64_t B, int y
   a.ytype = yt;
   a.nchunks = static_cast<int>((K + kChunkW - 1) / kChunkW);
   a.skip_first = 0;
+  a.split_cps = 0;
+  a.split_off = 0;
   const int terms = (xt == GQ_F32) ? 3 : 1;
   const int64_t per_chunk = static_cast<int64_t>(terms) * a.B * kXStride;
   int win = static_cast<int>(kXSmemMax / per_chunk);
-  // batches above 8 keep all of x resident when it fits beside the ring at
-  // one CTA per SM, rather than reloading windows for every row group
-  if (a.B > 8 && per_chunk * a.nchunks <= kXSmemFree) win = a.nchunks;
+  // batches keep all of x resident when it fits beside the ring at one CTA
+  // per SM, rather than reloading windows for every row group: a CTA whose
+  // x needs more than the window budget runs one per SM either way
+  if (a.B >= kResidentMinB && per_chunk * a.nchunks <= kXSmemFree) win = a.nchunks;
   if (win < 1) win = 1;
   if (win > a.nchunks) win = a.nchunks;
   a.win = win;
@@ -912,6 +1110,28 @@ gq_status gemv_entry(const void* W, int64_t M, int64_t K, const void* x, int xt,
   cudaStream_t s = as_stream(stream);
   if (workspace && ws_bytes && !skip_first && i8_eligible(FMT, M, K, B, xt, W))
     return i8_gemv(W, M, K, x, y, yt, workspace, ws_bytes, pdl, dev_status, s);
+  if (B > 1 && !skip_first && a.win < a.nchunks) {
+    // x does not fit beside the ring: split K over a cluster of up to 8 CTAs
+    // whose slices of x do, rather than reload windows for every row group
+    const int terms = (xt == GQ_F32) ? 3 : 1;
+    const int64_t per_chunk = static_cast<int64_t>(terms) * B * kXStride;
+    const int64_t room = kXSmemFree - 16 - static_cast<int64_t>(split_extra(B <= 8 ? 1 : 2));
+    const int cps_max = static_cast<int>(room / per_chunk);
+    const int cluster = cps_max >= 1 ? (a.nchunks + cps_max - 1) / cps_max : 0;
+    if (cluster >= 2 && cluster <= 8) {
+      GemvArgs sa = a;
+      sa.split_cps = (a.nchunks + cluster - 1) / cluster;  // every rank gets a chunk
+      sa.win = sa.split_cps;
+      bool launched = false;
+      gq_status st = GQ_OK;
+      switch (xt) {
+        case GQ_F16: st = dispatch_split<FMT, XT_F16>(sa, cluster, !misaligned16(W), s, pdl, launched); break;
+        case GQ_BF16: st = dispatch_split<FMT, XT_BF16>(sa, cluster, !misaligned16(W), s, pdl, launched); break;
+        default: st = dispatch_split<FMT, XT_F32>(sa, cluster, !misaligned16(W), s, pdl, launched); break;
+      }
+      if (launched) return st;
+    }
+  }
   return dispatch_xt<FMT>(a, NoTable{0}, xt, !misaligned16(W), s, pdl);
 }
 

@@ -155,7 +155,11 @@ GQ_API gq_status gq_dequantize_ksb(const void* q, int64_t n, float* out, void* s
  *   B: 1..8 (0 launches nothing).
  * Arithmetic: products of the exact decoded weights with the exact inputs
  * (fp32 x is split exactly into three bfloat16 terms), accumulated in fp32,
- * rounded once to y_dtype.
+ * rounded once to y_dtype.  When the B activation rows do not fit in one
+ * SM's shared memory beside the weight pipeline (e.g. B >= 6 at K = 11008
+ * with fp16 x), K is split over a thread-block cluster of 2..8 CTAs, each
+ * holding its slice of x; their fp32 partial sums are added in rank order,
+ * so results still do not depend on scheduling.
  * workspace / ws_bytes: optional caller-owned device scratch of at least
  *   gq_gemv_workspace_bytes(...) bytes (a size that does not depend on M or
  *   K), 256-byte aligned, all zero before its first use.  When that size is

@@ -118,6 +118,9 @@ def test_gemm_split_shapes(M, K, B):
     (Q40, 4096, 4096, 16, torch.float32),
     (KSB, 1000, 4096, 12, torch.float16),
     (Q40, 17, 8192, 11, torch.float32),
+    (Q40, 4096, 11008, 16, torch.float32),   # x beside the ring would need 399 KB:
+    (KSB, 1000, 11008, 12, torch.float16),   # K split over clusters of 3 CTAs
+    (Q40, 40, 16384, 16, torch.bfloat16),    # ... and of 4 CTAs
 ])
 def test_gemm_warp_mma_batches(fmt, M, K, B, ydt):
     # batches 9..16 take two n8 tiles of the warp MMA (every code decoded once

@@ -88,10 +88,45 @@ def test_batches_and_dtypes(B, xdt):
 
 
 def test_wide_batch_window():
-    # B=8 with K=11008: the activations do not fit shared memory at once and
-    # are streamed in windows
-    check(Q40, 64, 11008, 8, torch.float32, torch.float32)
-    check(KSB, 48, 11008, 8, torch.float16, torch.float32)
+    # fp32 activations of 8 rows at K = 20480 (ten 2048-weight chunks): a
+    # chunk of x alone fills the shared memory left beside the ring, so a
+    # K split would need more than 8 CTAs per cluster; x is streamed in
+    # windows instead
+    check(Q40, 40, 20480, 8, torch.float32, torch.float32)
+    check(KSB, 24, 20480, 8, torch.float32, torch.float16, gen="logstd")
+
+
+# Batches whose activations do not fit beside the ring: K is split over a
+# cluster of 2..8 CTAs, each with its slice of x resident, the partial sums
+# added in rank order through distributed shared memory.
+@pytest.mark.parametrize("fmt,M,K,B,xdt,ydt", [
+    (Q40, 4096, 11008, 8, torch.float16, torch.float16),   # 2 CTAs, 3 chunks each
+    (KSB, 300, 11008, 8, torch.float16, torch.float32),    # unaligned rows
+    (Q40, 300, 11008, 6, torch.bfloat16, torch.bfloat16),
+    (KSB, 129, 11008, 7, torch.float16, torch.float16),
+    (Q40, 64, 11008, 8, torch.float32, torch.float32),     # 6 CTAs, one chunk each
+    (KSB, 48, 11008, 8, torch.float16, torch.float32),
+    (KSB, 33, 16384, 8, torch.float16, torch.float16),     # 2 CTAs, 4 chunks each
+    (Q40, 17, 16384, 2, torch.float32, torch.float32),
+    (Q40, 1, 11008, 8, torch.float16, torch.float32),      # one row
+    (Q40, 7, 16448, 5, torch.float32, torch.float32),      # ragged last chunk, 5 CTAs
+])
+@pytest.mark.parametrize("flags", [0, 1])
+def test_k_split_over_cluster(fmt, M, K, B, xdt, ydt, flags):
+    check(fmt, M, K, B, xdt, ydt, gen="gauss" if fmt == Q40 else "logstd", flags=flags)
+
+
+def test_k_split_deterministic():
+    # rank 0 adds the other ranks' sums in rank order: repeated calls agree
+    # bit for bit
+    M, K, B = 1000, 11008, 8
+    q = torch.from_numpy(packed(KSB, M, K)).cuda()
+    x = synth.activations(B, K, seed=3, dtype=torch.float16).cuda()
+    ys = [gq.gq_gemv_ksb(q, M, K, x, y_dtype=torch.float32, flags=gq.GQ_GEMV_PDL)
+          for _ in range(4)]
+    torch.cuda.synchronize()
+    for y in ys[1:]:
+        assert torch.equal(y, ys[0])
 
 
 def test_k_zero_writes_zeros():
