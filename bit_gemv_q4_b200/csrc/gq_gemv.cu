@@ -538,13 +538,8 @@ __device__ void load_x_window(uint8_t* xs, const void* x, int64_t K, int B, int 
   }
 }
 
-// SPLIT: the CTAs of a cluster share each row group, CTA rank q taking the
-// chunks [q * split_cps, (q + 1) * split_cps) of every row with its slice of
-// x resident; rank 0 adds the other ranks' partial sums, in rank order, read
-// from their shared memory, and stores y.  A slice of x fills more than half
-// of the shared memory, so these CTAs run one per SM.
-template <int FMT, int XT, int NT, bool ALIGNED, class Tbl, bool SPLIT = false>
-__global__ void __launch_bounds__(kThreads, SPLIT ? 1 : GQ_GEMV_MINB)
+template <int FMT, int XT, int NT, bool ALIGNED, class Tbl>
+__global__ void __launch_bounds__(kThreads, GQ_GEMV_MINB)
     gemv_kernel(const GemvArgs a, const __grid_constant__ Tbl tbl) {
   constexpr int kBlkW = Fmt<FMT>::kBlkW, kBlkB = Fmt<FMT>::kBlkB;
   constexpr int kTerms = (XT == XT_F32) ? 3 : 1;
@@ -560,29 +555,10 @@ __global__ void __launch_bounds__(kThreads, SPLIT ? 1 : GQ_GEMV_MINB)
   uint64_t* empty = full + kStages;
   uint64_t* cbar = empty + kStages;  // consumer-group barrier (bounded waits)
   int* abort_flag = reinterpret_cast<int*>(cbar + 1);
-  // SPLIT exchange: every rank leaves its partial sums of group gi in its
-  // xred slot gi % kSplitSlots; part_full[p] (rank 0) completes when every
-  // lane of every other rank has done so, part_free[p] (other ranks) when
-  // rank 0's lanes have read them.  Rank 0 adds up a group one group later,
-  // so that its wait rarely holds up its own pipeline.
-  uint64_t* part_full = reinterpret_cast<uint64_t*>(smem + a.split_off);
-  uint64_t* part_free = part_full + kSplitSlots;
-  float* xred = reinterpret_cast<float*>(part_free + kSplitSlots);  // [slots][32][acc_len(NT)]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nblk_row = static_cast<int>(a.K / kBlkW);
   const int nfull = nblk_row / kBlkPerChunk;  // chunks with every block present
-  // this CTA's chunks of a row and its row groups g_first, g_first + g_step, ...
-  int c_begin = 0, c_end = a.nchunks, g_first = blockIdx.x, g_step = gridDim.x;
-  uint32_t rank = 0, nrank = 1;
-  if constexpr (SPLIT) {
-    rank = cluster_ctarank();
-    nrank = cluster_nctarank();
-    c_begin = static_cast<int>(rank) * a.split_cps;
-    c_end = min(a.nchunks, c_begin + a.split_cps);
-    g_first = static_cast<int>(cluster_id_x());
-    g_step = static_cast<int>(cluster_count_x());
-  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -590,18 +566,10 @@ __global__ void __launch_bounds__(kThreads, SPLIT ? 1 : GQ_GEMV_MINB)
       mbar_init(&empty[s], kConsumers);
     }
     mbar_init(cbar, kConsumers);
-    if constexpr (SPLIT) {
-      for (int p = 0; p < kSplitSlots; ++p) {
-        mbar_init(&part_full[p], 32 * (nrank - 1));
-        mbar_init(&part_free[p], 32);
-      }
-    }
     *abort_flag = 0;
     fence_barrier_init();
   }
   __syncthreads();
-  // every CTA's barriers exist before any other CTA of the cluster arrives on them
-  if constexpr (SPLIT) cluster_sync_all();
   pdl_launch_dependents();
 
   if (warp == 0) {
@@ -613,14 +581,13 @@ __global__ void __launch_bounds__(kThreads, SPLIT ? 1 : GQ_GEMV_MINB)
     bool ok = true;
     const uint32_t tail_bytes = static_cast<uint32_t>((nblk_row - nfull * kBlkPerChunk) * kBlkB);
     int pmi = 0;  // matrix cursor
-    for (int g = g_first; g < a.ngroups && ok; g += g_step) {
+    for (int g = blockIdx.x; g < a.ngroups && ok; g += gridDim.x) {
       const Unit un = unit_of(a, tbl, g, pmi);
       const int64_t m0 = un.m0;
       const bool row_ok = lane < kRows && m0 + lane < un.M;
       uintptr_t src = reinterpret_cast<uintptr_t>(un.W) +
-                      static_cast<uintptr_t>((m0 + (row_ok ? lane : 0)) * a.rowbytes +
-                                             static_cast<int64_t>(c_begin) * kChunkBytes);
-      for (int c = c_begin; c < c_end; ++c, ++issued, src += kChunkBytes) {
+                      static_cast<uintptr_t>((m0 + (row_ok ? lane : 0)) * a.rowbytes);
+      for (int c = 0; c < a.nchunks; ++c, ++issued, src += kChunkBytes) {
         if (!mbar_wait(&empty[s], ph ^ 1u, a.budget) ||
             *reinterpret_cast<volatile int*>(abort_flag)) {
           ok = false;
@@ -669,8 +636,6 @@ __global__ void __launch_bounds__(kThreads, SPLIT ? 1 : GQ_GEMV_MINB)
         }
       }
     }
-    // no CTA of the cluster leaves while another may still read its memory
-    if constexpr (SPLIT) cluster_sync_all();
     return;
   }
 
@@ -700,9 +665,9 @@ __global__ void __launch_bounds__(kThreads, SPLIT ? 1 : GQ_GEMV_MINB)
 
   pdl_wait();  // the preceding grid has finished: x is ready, y may be written
 
-  const bool x_resident = (a.win >= c_end - c_begin);
+  const bool x_resident = (a.win >= a.nchunks);
   if (x_resident) {
-    load_x_window<XT>(xs, a.x, a.K, a.B, c_begin, a.win, term_stride, ctid);
+    load_x_window<XT>(xs, a.x, a.K, a.B, 0, a.win, term_stride, ctid);
     ok = group_sync();
   }
   const uint32_t x_chunk = static_cast<uint32_t>(a.B * kXStride);
@@ -710,86 +675,25 @@ __global__ void __launch_bounds__(kThreads, SPLIT ? 1 : GQ_GEMV_MINB)
   // n8 tile 1 holds batch rows 8..15: this lane's row there, relative to tile 0
   const uint32_t xt1 = static_cast<uint32_t>((min(8 + r, a.B - 1) - bsel) * kXStride);
 
-  constexpr int kTiles = NT > 1 ? NT : 1;
-  // y at rows m0 + r and m0 + r + 8 of the batch columns this lane holds
-  // (NT = 0: lane t = 0 holds row r, lane t = 1 row r + 8, see scale_acc)
-  auto store_rows = [&](const float* v, void* y, int64_t M, int64_t m0) {
-    const int64_t ra = m0 + r, rbw = m0 + r + 8;
-    if constexpr (NT == 0) {
-      const int64_t row = (t == 0) ? ra : rbw;
-      if (t < 2 && row < M) store_elem(y, row, v[0], a.ytype);
-    } else {
-#pragma unroll
-      for (int n = 0; n < kTiles; ++n) {
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int col = 8 * n + 2 * t + i;
-          if (col < a.B) {
-            if (ra < M) store_elem(y, col * M + ra, v[4 * n + i], a.ytype);
-            if (rbw < M) store_elem(y, col * M + rbw, v[4 * n + 2 + i], a.ytype);
-          }
-        }
-      }
-    }
-  };
-  // SPLIT, rank 0, warp 0: add up group gj (row group gg) from every rank's
-  // slot, in rank order, and store it.  Each lane reads and releases only
-  // its own entries.
-  auto split_finish = [&](int gj, int gg) -> bool {
-    const int p = gj % kSplitSlots;
-    if (!__all_sync(0xFFFFFFFFu, mbar_wait_cluster(&part_full[p],
-                                                   static_cast<uint32_t>(gj / kSplitSlots) & 1u,
-                                                   a.budget)))
-      return false;
-    const float4* slot = reinterpret_cast<const float4*>(xred) + (p * 32 + lane) * kTiles;
-    float v[acc_len(NT)];
-#pragma unroll
-    for (int n = 0; n < kTiles; ++n) {
-      const float4 o = slot[n];
-      v[4 * n + 0] = o.x;
-      v[4 * n + 1] = o.y;
-      v[4 * n + 2] = o.z;
-      v[4 * n + 3] = o.w;
-    }
-    const uint32_t sa = smem_addr(slot);
-    for (uint32_t q = 1; q < nrank; ++q) {
-#pragma unroll
-      for (int n = 0; n < kTiles; ++n) {
-        const float4 w = ld_cluster_f4(sa + 16u * n, q);
-        v[4 * n + 0] += w.x;
-        v[4 * n + 1] += w.y;
-        v[4 * n + 2] += w.z;
-        v[4 * n + 3] += w.w;
-      }
-    }
-    for (uint32_t q = 1; q < nrank; ++q) mbar_arrive_remote(&part_free[p], q);
-    store_rows(v, a.y, a.M, static_cast<int64_t>(gg) * kRows);
-    return true;
-  };
-
   int s = 0;        // stage of the next use
   uint32_t ph = 0;  // its phase parity
   int gi = 0;       // groups done by this CTA
   int cmi = 0;  // matrix cursor
-  for (int g = g_first; g < a.ngroups && ok; g += g_step, ++gi) {
+  for (int g = blockIdx.x; g < a.ngroups && ok; g += gridDim.x, ++gi) {
     const Unit un = unit_of(a, tbl, g, cmi);
     const int64_t m0 = un.m0;
     float acc[acc_len(NT)];
 #pragma unroll
     for (int q = 0; q < acc_len(NT); ++q) acc[q] = 0.f;
-    // offset of row r's (and r+8's) first byte of chunk c_begin inside its
-    // 16-byte granule
-    const int64_t cb_off = static_cast<int64_t>(c_begin) * kChunkBytes;
+    // offset of row r's (and r+8's) first byte inside its 16-byte granule
     uint32_t off0 = static_cast<uint32_t>(
-        (reinterpret_cast<uintptr_t>(un.W) + static_cast<uintptr_t>((m0 + r) * a.rowbytes + cb_off)) &
-        15u);
+        (reinterpret_cast<uintptr_t>(un.W) + static_cast<uintptr_t>((m0 + r) * a.rowbytes)) & 15u);
     uint32_t off1 = static_cast<uint32_t>(
-        (reinterpret_cast<uintptr_t>(un.W) +
-         static_cast<uintptr_t>((m0 + r + 8) * a.rowbytes + cb_off)) &
+        (reinterpret_cast<uintptr_t>(un.W) + static_cast<uintptr_t>((m0 + r + 8) * a.rowbytes)) &
         15u);
     uint32_t xw = x_lane;
     int cw_in_win = 0;
-    for (int c = c_begin; c < c_end; ++c) {
+    for (int c = 0; c < a.nchunks; ++c) {
       if (!x_resident && cw_in_win == 0) {
         if (!group_sync()) { ok = false; break; }
         load_x_window<XT>(xs, a.x, a.K, a.B, c, a.win, term_stride, ctid);
@@ -840,6 +744,7 @@ __global__ void __launch_bounds__(kThreads, SPLIT ? 1 : GQ_GEMV_MINB)
 
     // reduce the consumer warps' partial sums (double-buffered by group
     // parity, so one barrier per group suffices), then store
+    constexpr int kTiles = NT > 1 ? NT : 1;
     float4* rb = reinterpret_cast<float4*>(red) + (gi & 1) * kConsumers * 32 * kTiles;
 #pragma unroll
     for (int n = 0; n < kTiles; ++n)
@@ -861,42 +766,345 @@ __global__ void __launch_bounds__(kThreads, SPLIT ? 1 : GQ_GEMV_MINB)
           s4[4 * n + 3] += v.w;
         }
       }
-      if constexpr (SPLIT) {
-        const int p = gi % kSplitSlots;
-        float4* slot = reinterpret_cast<float4*>(xred) + (p * 32 + lane) * kTiles;
-        // rank 0 has read what this slot held kSplitSlots groups ago (its own
-        // slot it read itself, one group after writing it)
-        if (rank != 0 && gi >= kSplitSlots &&
-            !__all_sync(0xFFFFFFFFu,
-                        mbar_wait_cluster(&part_free[p],
-                                          static_cast<uint32_t>(gi / kSplitSlots - 1) & 1u,
-                                          a.budget))) {
-          ok = false;
-        } else {
-#pragma unroll
-          for (int n = 0; n < kTiles; ++n)
-            slot[n] = make_float4(s4[4 * n], s4[4 * n + 1], s4[4 * n + 2], s4[4 * n + 3]);
-          if (rank != 0) mbar_arrive_remote(&part_full[p], 0);
-          // the previous group's parts are in, or about to be
-          if (rank == 0 && gi >= 1 && !split_finish(gi - 1, g - g_step)) ok = false;
-        }
+      const int64_t ra = m0 + r, rbw = m0 + r + 8;
+      if constexpr (NT == 0) {
+        // lane t = 0 holds row r, lane t = 1 row r + 8 (scale_acc)
+        const int64_t row = (t == 0) ? ra : rbw;
+        if (t < 2 && row < un.M) store_elem(un.y, row, s4[0], a.ytype);
       } else {
-        store_rows(s4, un.y, un.M, m0);
+#pragma unroll
+        for (int n = 0; n < kTiles; ++n) {
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int col = 8 * n + 2 * t + i;
+            if (col < a.B) {
+              if (ra < un.M) store_elem(un.y, col * un.M + ra, s4[4 * n + i], a.ytype);
+              if (rbw < un.M) store_elem(un.y, col * un.M + rbw, s4[4 * n + 2 + i], a.ytype);
+            }
+          }
+        }
       }
     }
-  }
-  // SPLIT: rank 0 adds up its last group
-  if constexpr (SPLIT) {
-    if (ok && cw == 0 && rank == 0 && gi >= 1 && !split_finish(gi - 1, g_first + (gi - 1) * g_step))
-      ok = false;
   }
 
   if (!ok && lane == 0) {
     report(a.dev_status, GQ_DEV_TIMEOUT);
     *reinterpret_cast<volatile int*>(abort_flag) = 1;
   }
+}
+
+// One matrix with K split over a thread-block cluster.  The CTAs of a
+// cluster share each of the cluster's row groups g = clusterid,
+// clusterid + nclusters, ...: rank q takes chunks [q * split_cps,
+// (q + 1) * split_cps) of every row, with its slice of x resident (the host
+// sizes the slice to fit).  At the end of a group every rank leaves its fp32
+// sums in slot gi % kSplitSlots of its own shared memory; rank 0 adds them
+// up one group later, in rank order, reading the other ranks' slots through
+// distributed shared memory, and stores y.  A slice of x fills more than half
+// of the shared memory, so these CTAs run one per SM.  Apart from the chunk
+// range, the group sequence and the exchange, each step is gemv_kernel's.
+template <int FMT, int XT, int NT, bool ALIGNED>
+__global__ void __launch_bounds__(kThreads, 1) gemv_split_kernel(const GemvArgs a) {
+  constexpr int kBlkW = Fmt<FMT>::kBlkW, kBlkB = Fmt<FMT>::kBlkB;
+  constexpr int kTerms = (XT == XT_F32) ? 3 : 1;
+  constexpr int kBlkPerChunk = kChunkW / kBlkW;
+  constexpr int kChunkBytes = kBlkPerChunk * kBlkB;
+  constexpr int kTiles = NT > 1 ? NT : 1;
+
+  uint8_t* stages = smem;
+  uint8_t* xs = smem + kStages * kStageBytes;
+  const uint32_t term_stride = static_cast<uint32_t>(a.win * a.B * kXStride);
+  // [2][kConsumers][32][acc_len(NT)]
+  float* red = reinterpret_cast<float*>(xs + kTerms * term_stride);
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + 2 * kConsumers * 32 * acc_len(NT));
+  uint64_t* empty = full + kStages;
+  uint64_t* cbar = empty + kStages;  // consumer-group barrier (bounded waits)
+  int* abort_flag = reinterpret_cast<int*>(cbar + 1);
+  // the exchange: part_full[p] (used in rank 0) completes when every lane of
+  // every other rank has left its sums of a group in its slot p; part_free[p]
+  // (other ranks) when rank 0's lanes have read them
+  uint64_t* part_full = reinterpret_cast<uint64_t*>(smem + a.split_off);
+  uint64_t* part_free = part_full + kSplitSlots;
+  float* xred = reinterpret_cast<float*>(part_free + kSplitSlots);  // [slots][32][acc_len(NT)]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nblk_row = static_cast<int>(a.K / kBlkW);
+  const int nfull = nblk_row / kBlkPerChunk;  // chunks with every block present
+  const uint32_t rank = cluster_ctarank(), nrank = cluster_nctarank();
+  const int c_begin = static_cast<int>(rank) * a.split_cps;
+  const int c_end = min(a.nchunks, c_begin + a.split_cps);
+  const int g_first = static_cast<int>(cluster_id_x());
+  const int g_step = static_cast<int>(cluster_count_x());
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumers);
+    }
+    mbar_init(cbar, kConsumers);
+    for (int p = 0; p < kSplitSlots; ++p) {
+      mbar_init(&part_full[p], 32 * (nrank - 1));
+      mbar_init(&part_free[p], 32);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // every CTA's barriers exist before any other CTA of the cluster arrives on them
+  cluster_sync_all();
+  pdl_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    const uint64_t pol = policy_evict_first();
+    int issued = 0;      // stage uses issued so far (all groups)
+    int s = 0;           // stage of the next use
+    uint32_t ph = 0;     // its phase parity
+    bool ok = true;
+    const uint32_t tail_bytes = static_cast<uint32_t>((nblk_row - nfull * kBlkPerChunk) * kBlkB);
+    for (int g = g_first; g < a.ngroups && ok; g += g_step) {
+      const int64_t m0 = static_cast<int64_t>(g) * kRows;
+      const bool row_ok = lane < kRows && m0 + lane < a.M;
+      uintptr_t src = reinterpret_cast<uintptr_t>(a.W) +
+                      static_cast<uintptr_t>((m0 + (row_ok ? lane : 0)) * a.rowbytes +
+                                             static_cast<int64_t>(c_begin) * kChunkBytes);
+      for (int c = c_begin; c < c_end; ++c, ++issued, src += kChunkBytes) {
+        if (!mbar_wait(&empty[s], ph ^ 1u, a.budget) ||
+            *reinterpret_cast<volatile int*>(abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint32_t nbytes = (c < nfull) ? static_cast<uint32_t>(kChunkBytes) : tail_bytes;
+        uint32_t len = 0;
+        uintptr_t lo = 0;
+        if (row_ok) {
+          lo = src & ~static_cast<uintptr_t>(15);
+          len = static_cast<uint32_t>(((src + nbytes + 15) & ~static_cast<uintptr_t>(15)) - lo);
+        }
+        uint32_t total = len;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xFFFFFFFFu, total, o);
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], total);
+        __syncwarp();
+        if (len)
+          bulk_g2s(stages + s * kStageBytes + lane * kPitch, reinterpret_cast<const void*>(lo), len,
+                   &full[s], pol);
+        if (++s == kStages) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      report(a.dev_status, GQ_DEV_TIMEOUT);
+      *reinterpret_cast<volatile int*>(abort_flag) = 1;
+    }
+    // Drain: every issued copy must land before this CTA's shared memory is
+    // released, whatever the consumers did.
+    if (lane == 0) {
+      for (int u = max(0, issued - kStages); u < issued; ++u) {
+        if (!mbar_wait(&full[u % kStages], static_cast<uint32_t>(u / kStages) & 1u, a.budget)) {
+          report(a.dev_status, GQ_DEV_TIMEOUT);
+          break;
+        }
+      }
+    }
+    // no CTA of the cluster leaves while another may still read its memory
+    cluster_sync_all();
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int cw = warp - 1;                // consumer index, also its share of a chunk
+  const int ctid = threadIdx.x - 32;      // 0 .. 32 * kConsumers - 1
+  const int r = lane >> 2, t = lane & 3;  // fragment row group / thread in group
+  const int bsel = min(r, a.B - 1);       // batch column this lane's B fragment reads
+  bool ok = true;
+  uint32_t cphase = 0;
+  auto group_sync = [&]() -> bool {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(cbar);
+    const bool done = mbar_wait(cbar, cphase & 1u, a.budget);
+    ++cphase;
+    return done;
+  };
+
+  // this warp's share of a ragged last chunk
+  int tail_valid;
+  if constexpr (FMT == GQ_FMT_Q4_0)
+    tail_valid = min(max(nblk_row - nfull * kBlkPerChunk - kSubPerWarp * cw, 0), kSubPerWarp);
+  else
+    tail_valid = ((cw * kSubPerWarp) >> 3) < nblk_row - nfull * kBlkPerChunk;
+
+  pdl_wait();  // the preceding grid has finished: x is ready, y may be written
+
+  // this rank's slice of x, resident for the whole kernel
+  load_x_window<XT>(xs, a.x, a.K, a.B, c_begin, a.win, term_stride, ctid);
+  ok = group_sync();
+  const uint32_t x_chunk = static_cast<uint32_t>(a.B * kXStride);
+  const uint32_t x_lane = static_cast<uint32_t>(xs - smem) + bsel * kXStride + t * 16;
+  // n8 tile 1 holds batch rows 8..15: this lane's row there, relative to tile 0
+  const uint32_t xt1 = static_cast<uint32_t>((min(8 + r, a.B - 1) - bsel) * kXStride);
+
+  // rank 0, warp 0: add up group gj (row group gg) from every rank's slot,
+  // in rank order, and store it; each lane reads and releases only its own
+  // entries
+  auto finish = [&](int gj, int gg) -> bool {
+    const int p = gj % kSplitSlots;
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait_cluster(&part_full[p],
+                                                   static_cast<uint32_t>(gj / kSplitSlots) & 1u,
+                                                   a.budget)))
+      return false;
+    const float4* slot = reinterpret_cast<const float4*>(xred) + (p * 32 + lane) * kTiles;
+    float v[acc_len(NT)];
+#pragma unroll
+    for (int n = 0; n < kTiles; ++n) {
+      const float4 o = slot[n];
+      v[4 * n + 0] = o.x;
+      v[4 * n + 1] = o.y;
+      v[4 * n + 2] = o.z;
+      v[4 * n + 3] = o.w;
+    }
+    const uint32_t sa = smem_addr(slot);
+    for (uint32_t q = 1; q < nrank; ++q) {
+#pragma unroll
+      for (int n = 0; n < kTiles; ++n) {
+        const float4 w = ld_cluster_f4(sa + 16u * n, q);
+        v[4 * n + 0] += w.x;
+        v[4 * n + 1] += w.y;
+        v[4 * n + 2] += w.z;
+        v[4 * n + 3] += w.w;
+      }
+    }
+    for (uint32_t q = 1; q < nrank; ++q) mbar_arrive_remote(&part_free[p], q);
+    const int64_t ra = static_cast<int64_t>(gg) * kRows + r, rbw = ra + 8;
+#pragma unroll
+    for (int n = 0; n < kTiles; ++n) {
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int col = 8 * n + 2 * t + i;
+        if (col < a.B) {
+          if (ra < a.M) store_elem(a.y, col * a.M + ra, v[4 * n + i], a.ytype);
+          if (rbw < a.M) store_elem(a.y, col * a.M + rbw, v[4 * n + 2 + i], a.ytype);
+        }
+      }
+    }
+    return true;
+  };
+
+  int s = 0;        // stage of the next use
+  uint32_t ph = 0;  // its phase parity
+  int gi = 0;       // groups done by this CTA
+  for (int g = g_first; g < a.ngroups && ok; g += g_step, ++gi) {
+    const int64_t m0 = static_cast<int64_t>(g) * kRows;
+    float acc[acc_len(NT)];
+#pragma unroll
+    for (int q = 0; q < acc_len(NT); ++q) acc[q] = 0.f;
+    // offset of row r's (and r+8's) first byte of chunk c_begin inside its
+    // 16-byte granule
+    const int64_t cb_off = static_cast<int64_t>(c_begin) * kChunkBytes;
+    uint32_t off0 = static_cast<uint32_t>(
+        (reinterpret_cast<uintptr_t>(a.W) + static_cast<uintptr_t>((m0 + r) * a.rowbytes + cb_off)) &
+        15u);
+    uint32_t off1 = static_cast<uint32_t>(
+        (reinterpret_cast<uintptr_t>(a.W) +
+         static_cast<uintptr_t>((m0 + r + 8) * a.rowbytes + cb_off)) &
+        15u);
+    uint32_t xw = x_lane;
+    for (int c = c_begin; c < c_end; ++c) {
+      if (!mbar_wait(&full[s], ph, a.budget) || *reinterpret_cast<volatile int*>(abort_flag)) {
+        ok = false;
+        break;
+      }
+      const uint32_t stg = static_cast<uint32_t>(s * kStageBytes);  // stages start at offset 0
+      const bool whole = c < nfull;
+      if constexpr (FMT == GQ_FMT_Q4_0) {
+        const int nvalid = whole ? kSubPerWarp : tail_valid;
+        if constexpr (ALIGNED) {
+          q40_chunk<XT, NT, true>(acc, stg + r * kPitch, stg + (r + 8) * kPitch, xw,
+                                  term_stride, xt1, cw, t, nvalid);
+        } else {
+          q40_chunk<XT, NT, false>(acc, stg + r * kPitch + off0, stg + (r + 8) * kPitch + off1,
+                                   xw, term_stride, xt1, cw, t, nvalid);
+        }
+      } else {
+        if (whole || tail_valid) {
+          const uint32_t p0 = stg + r * kPitch + off0, p1 = stg + (r + 8) * kPitch + off1;
+          if constexpr (ALIGNED) {
+            if (((cw * kSubPerWarp) >> 3) & 1)
+              ksb_chunk<XT, NT, 0>(acc, p0, p1, xw, term_stride, xt1, cw, t);
+            else
+              ksb_chunk<XT, NT, 2>(acc, p0, p1, xw, term_stride, xt1, cw, t);
+          } else {
+            ksb_chunk<XT, NT, -1>(acc, p0, p1, xw, term_stride, xt1, cw, t);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (++s == kStages) {
+        s = 0;
+        ph ^= 1u;
+      }
+      off0 = (off0 + kChunkBytes) & 15u;
+      off1 = (off1 + kChunkBytes) & 15u;
+      xw += x_chunk;
+    }
+    if (!ok) break;
+
+    // the consumer warps' sums meet in the reduction buffer (double-buffered
+    // by group parity), then warp 0 hands this CTA's part to the exchange
+    float4* rb = reinterpret_cast<float4*>(red) + (gi & 1) * kConsumers * 32 * kTiles;
+#pragma unroll
+    for (int n = 0; n < kTiles; ++n)
+      rb[(cw * 32 + lane) * kTiles + n] =
+          make_float4(acc[4 * n], acc[4 * n + 1], acc[4 * n + 2], acc[4 * n + 3]);
+    if (!group_sync()) { ok = false; break; }
+    if (cw == 0) {
+      float s4[acc_len(NT)];
+#pragma unroll
+      for (int q = 0; q < acc_len(NT); ++q) s4[q] = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumers; ++w) {
+#pragma unroll
+        for (int n = 0; n < kTiles; ++n) {
+          const float4 v = rb[(w * 32 + lane) * kTiles + n];
+          s4[4 * n + 0] += v.x;
+          s4[4 * n + 1] += v.y;
+          s4[4 * n + 2] += v.z;
+          s4[4 * n + 3] += v.w;
+        }
+      }
+      const int p = gi % kSplitSlots;
+      float4* slot = reinterpret_cast<float4*>(xred) + (p * 32 + lane) * kTiles;
+      // rank 0 has read what this slot held kSplitSlots groups ago (its own
+      // slot it read itself, one group after writing it)
+      if (rank != 0 && gi >= kSplitSlots &&
+          !__all_sync(0xFFFFFFFFu,
+                      mbar_wait_cluster(&part_free[p],
+                                        static_cast<uint32_t>(gi / kSplitSlots - 1) & 1u,
+                                        a.budget))) {
+        ok = false;
+      } else {
+#pragma unroll
+        for (int n = 0; n < kTiles; ++n)
+          slot[n] = make_float4(s4[4 * n], s4[4 * n + 1], s4[4 * n + 2], s4[4 * n + 3]);
+        if (rank != 0) mbar_arrive_remote(&part_full[p], 0);
+        // the previous group's parts are in, or about to be
+        if (rank == 0 && gi >= 1 && !finish(gi - 1, g - g_step)) ok = false;
+      }
+    }
+  }
+  // rank 0 adds up its last group
+  if (ok && cw == 0 && rank == 0 && gi >= 1 && !finish(gi - 1, g_first + (gi - 1) * g_step))
+    ok = false;
+
+  if (!ok && lane == 0) {
+    report(a.dev_status, GQ_DEV_TIMEOUT);
+    *reinterpret_cast<volatile int*>(abort_flag) = 1;
+  }
   // no CTA of the cluster leaves while another may still read its memory
-  if constexpr (SPLIT) cluster_sync_all();
+  cluster_sync_all();
 }
 
 size_t gemv_smem_bytes(int B, int terms, int win) {
@@ -956,7 +1164,7 @@ template <int FMT, int XT, int NT, bool ALIGNED>
 gq_status launch_gemv_split(GemvArgs a, int cluster, cudaStream_t stream, bool pdl,
                             bool& launched) {
   constexpr int kTerms = (XT == XT_F32) ? 3 : 1;
-  auto kern = gemv_kernel<FMT, XT, NT, ALIGNED, NoTable, true>;
+  auto kern = gemv_split_kernel<FMT, XT, NT, ALIGNED>;
   const size_t base = (gemv_smem_bytes(a.B, kTerms, a.win) + 15) & ~static_cast<size_t>(15);
   a.split_off = static_cast<uint32_t>(base);
   const size_t smem = base + split_extra(NT);
@@ -1003,7 +1211,7 @@ gq_status launch_gemv_split(GemvArgs a, int cluster, cudaStream_t stream, bool p
   }
   const int nclusters = a.ngroups < max_clusters ? a.ngroups : max_clusters;
   return launch_cluster(kern, dim3(static_cast<unsigned>(nclusters * cluster)), dim3(kThreads),
-                        smem, stream, pdl, static_cast<unsigned>(cluster), a, NoTable{0});
+                        smem, stream, pdl, static_cast<unsigned>(cluster), a);
 }
 
 template <int FMT, int XT>
