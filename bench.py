@@ -419,19 +419,28 @@ def extra_rows(gq, synth, dev, peak, bf16):
         Ts = [gq.gq_repack(fmt_code, qm, M, K) for qm, M, K in mats]
         ft = gq.gq_gemv_q4_0_tiled_grouped if fmt == "q4_0" else gq.gq_gemv_ksb_tiled_grouped
         mst = _graph_ms(lambda: ft(Ts, Ms, 4096, x, outs=outs, flags=gq.GQ_GEMV_PDL), 5)
+        # one grouped call per decoder layer (its 7 matrices), 32 calls chained with PDL
+        L = 7
+        msl = _graph_ms(lambda: [fg(Ws[i:i + L], Ms[i:i + L], 4096, x, outs=outs[i:i + L],
+                                    flags=gq.GQ_GEMV_PDL) for i in range(0, len(Ms), L)], 5)
+        mstl = _graph_ms(lambda: [ft(Ts[i:i + L], Ms[i:i + L], 4096, x, outs=outs[i:i + L],
+                                     flags=gq.GQ_GEMV_PDL) for i in range(0, len(Ms), L)], 5)
         g1, g2, g3 = (total / (t * 1e-3) / 1e9 for t in (ms, msg, mst))
+        g4, g5 = (total / (t * 1e-3) / 1e9 for t in (msl, mstl))
 
         def row(t, g):
             return {"ms": round(t, 3), "gbs": round(g, 1), "frac_of_peak": frac(g),
                     "matrices_per_s": round(224 / (t * 1e-3), 1)}
         ms_rows[fmt] = {"weight_bytes": total, "graph": row(ms, g1), "grouped": row(msg, g2),
-                        "grouped_tiled": row(mst, g3)}
+                        "grouped_tiled": row(mst, g3), "grouped_per_layer": row(msl, g4),
+                        "grouped_tiled_per_layer": row(mstl, g5)}
         del mats, Ws, Ts, outs
         torch.cuda.empty_cache()
     out["model_stream"] = dict(
         workload="32 layers x (4 x 4096x4096 + 3 x 11008x4096) = 224 batch-1 GEMVs, x fp16; "
                  "'graph': one CUDA graph of 224 PDL launches, 'grouped': one grouped call, "
-                 "'grouped_tiled': one grouped call on tiled storage "
+                 "'grouped_tiled': one grouped call on tiled storage; '*_per_layer': one "
+                 "grouped call per layer (7 matrices), 32 calls chained with PDL in one graph "
                  "(weight_bytes: the canonical bytes, the same for both layouts)",
         **ms_rows)
 
