@@ -52,15 +52,15 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # it null until it is captured again.
 TRAFFIC = {
     "canonical ksb 4096 11008": {"bytes": 24349440, "sources": {
-            "bit_gemv_q4_b200/csrc/gq_gemv.cu": "8159186c5dfe4c9660def7e2c5372672c04816e77aeee451d83624142609143e",
+            "bit_gemv_q4_b200/csrc/gq_gemv.cu": "b6737f175c04b0f93c608fece7df7fed31a2b2d12f0bed7bba5339b9ec20c40e",
             "bit_gemv_q4_b200/csrc/gq_gemv.h": "91b29c15fbd80ae3ad2435b203453a1ba1d4da29da52322e6e996adb97cd8ebe",
             "bit_gemv_q4_b200/csrc/gq_device.cuh": "dc4d0fc96908a38ffd15ae87b6aecb7f02d029f2b003e9cbdae6614ee1f5e7a2"}},
     "tiled q4_0 4096 11008": {"bytes": 25420800, "sources": {
-            "bit_gemv_q4_b200/csrc/gq_tiled.cu": "f94739c717d66ab0050bc9e7f62f740954cc5907f6b9d416c1707d0da967a633",
+            "bit_gemv_q4_b200/csrc/gq_tiled.cu": "ef9b0561deae33b7305288cce25dfd501156aa1738d446a4e783e86696996c40",
             "bit_gemv_q4_b200/csrc/gq_device.cuh": "dc4d0fc96908a38ffd15ae87b6aecb7f02d029f2b003e9cbdae6614ee1f5e7a2",
             "bit_gemv_q4_b200/csrc/gq_tc.cuh": "b15f28de0672760637e15afae0059536e9c3acc85b1737d0e290acd10794f382"}},
     "tiled ksb 4096 11008": {"bytes": 24364032, "sources": {
-            "bit_gemv_q4_b200/csrc/gq_tiled.cu": "f94739c717d66ab0050bc9e7f62f740954cc5907f6b9d416c1707d0da967a633",
+            "bit_gemv_q4_b200/csrc/gq_tiled.cu": "ef9b0561deae33b7305288cce25dfd501156aa1738d446a4e783e86696996c40",
             "bit_gemv_q4_b200/csrc/gq_device.cuh": "dc4d0fc96908a38ffd15ae87b6aecb7f02d029f2b003e9cbdae6614ee1f5e7a2",
             "bit_gemv_q4_b200/csrc/gq_tc.cuh": "b15f28de0672760637e15afae0059536e9c3acc85b1737d0e290acd10794f382"}},
 }

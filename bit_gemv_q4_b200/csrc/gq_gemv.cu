@@ -30,6 +30,10 @@
 //    per k-step); fp16 and bf16 activations use one.  Activations sit in
 //    shared memory in B-fragment order (one 16-byte load per lane per block)
 //    and are loaded once per CTA when they fit, else per window.
+//  * Batches whose activations do not fit beside the ring at one CTA per SM
+//    run gemv_split_kernel: K is split over a thread-block cluster of 2..8
+//    CTAs, each holding its slice of x, and rank 0 adds the ranks' fp32 sums
+//    in rank order through distributed shared memory.
 //  * Programmatic dependent launch: the producer streams W at once; consumers
 //    wait for the preceding grid before reading x or writing y.
 //  * Every wait is bounded; on expiry the kernel sets GQ_DEV_TIMEOUT, drains

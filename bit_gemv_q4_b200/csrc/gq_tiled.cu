@@ -43,6 +43,14 @@
 // warp keeps its share of a row in registers and leaves it in a shared
 // table; the shares of a batch of row groups are added at one barrier.
 //
+// Grouped form (gq_gemv_*_tiled_grouped).  Many tiled matrices that share K
+// and x go into one launch: their row groups are numbered back to back and a
+// table passed by value maps a group to its matrix.  A group's arithmetic
+// does not depend on the CTA that takes it, so each output equals the
+// single-matrix call's bit for bit.  This launch puts two CTAs on each SM
+// and always stages the first tiles in tensor memory, which measured fastest
+// on long grouped streams.
+//
 // Every wait is bounded (kWaitBudget cycles); on expiry the kernel ORs
 // GQ_DEV_TIMEOUT into the status word, lets its copies land, releases its
 // tensor memory and exits.
