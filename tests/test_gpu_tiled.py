@@ -276,3 +276,30 @@ def test_tiled_grouped_table_batches(fmt):
         assert int(st.item()) == 0
         assert_product_close(ys[0], Y, bound)
         assert torch.equal(ys[0], ys[1])
+
+
+@pytest.mark.parametrize("fmt", [Q40, KSB])
+def test_tiled_grouped_chained_layers(fmt):
+    # one grouped call per layer, three layers chained with PDL, so that each
+    # launch stages its first tiles (six tiles per row group at K = 11008,
+    # more than the ring holds) while the previous one still runs; every
+    # output equals the same call made alone, and one matrix is checked
+    # against the oracle
+    K = 11008
+    Ms = [256] * 4 + [688] * 3
+    qs = [[packed(fmt, M, K, seed=500 + 10 * l + i) for i, M in enumerate(Ms)] for l in range(3)]
+    Ts = [[tiled(fmt, q, M, K) for q, M in zip(ql, Ms)] for ql in qs]
+    x = synth.activations(1, K, seed=31, dtype=torch.float16)
+    xd = x.cuda()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ys = [grouped(fmt)(Tl, Ms, K, xd, y_dtype=torch.float32, flags=gq.GQ_GEMV_PDL, dev_status=st)
+          for Tl in Ts]
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for Tl, yl in zip(Ts, ys):
+        alone = grouped(fmt)(Tl, Ms, K, xd, y_dtype=torch.float32)
+        torch.cuda.synchronize()
+        for a, b in zip(yl, alone):
+            assert torch.equal(a, b)
+    Y, bound = oracle.gemm(fmt, qs[2][5], Ms[5], K, *x_for_oracle(x))
+    assert_product_close(ys[2][5], Y, bound)
