@@ -218,7 +218,9 @@ def test_concurrent_host_threads():
     # shared-memory sizes and kernel configurations) on their own streams at
     # once; every result equals the same call made alone
     import threading
-    cases = [(Q40, 4096, 4096, 1), (KSB, 300, 11008, 1), (Q40, 1000, 2048, 8), (KSB, 129, 4352, 3)]
+    # (the last case splits K over clusters of 2 CTAs)
+    cases = [(Q40, 4096, 4096, 1), (KSB, 300, 11008, 1), (Q40, 1000, 2048, 8), (KSB, 129, 4352, 3),
+             (KSB, 200, 11008, 8)]
     data = []
     for fmt, M, K, B in cases:
         q = torch.from_numpy(packed(fmt, M, K)).cuda()
